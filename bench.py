@@ -1,0 +1,496 @@
+"""Benchmark of the GDN / KDA token mixers on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Workloads (synthetic inputs, recipe in synth/):
+  gdn_prefill  GDN chunked prefill, B=1 H=32 T=4096 d=128 bf16       (default)
+  kda_prefill  KDA chunked prefill, same shapes, per-channel gates
+  decode_gdn   256 sequences x 32 heads, d=128, 512 one-token steps, GDN gates
+  decode_kda   same with KDA gates
+  kda_long     KDA prefill with a carried state, B=4 H=32 T=65536 d=128
+
+One step is one pass of the workload: one prefill call, or 512 decode calls.
+`value` is whole-job tokens/s (a token = one position of one sequence, all H
+heads) with inputs resident in HBM; `e2e` is the same through the public API
+with pinned host buffers copied in and results copied out inside the timed
+region.  Under torchrun each rank runs its own replica of the workload (the
+(sequence, head) chains are independent, so nothing is exchanged): weak
+scaling, time = max over ranks.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, device_inputs, slice_inputs  # noqa: E402
+
+METRIC = "GDN/KDA prefill tokens/s and decode tokens/s at 1 B200; % of roofline"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------------------
+# algorithmic work per workload
+# ----------------------------------------------------------------------------------------
+
+def algorithmic(w):
+    """(bytes, flops) of one pass of workload w, counted from the definition:
+    every input read once, every output written once; flops of the chunked form
+    at C=64 (2C(3 d_k + 2 d_v) + 6 d_k d_v per token-head, excluding the
+    triangular solve and the gate exponentials).  Decode counts the state bytes
+    (read + write) only, which is 99% of its traffic."""
+    esz = 2 if w.dtype == "bf16" else 4
+    th = w.B * w.T * w.H
+    state = w.B * w.H * w.dv * w.dk * 4
+    if w.decode:
+        return 2 * state * w.T, th * 6 * w.dk * w.dv
+    a_bytes = 4 * (w.dk if w.mixer == "kda" else 1)
+    per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
+    nbytes = th * per_th + state + (state if w.state == "randn" else 0)
+    C = 64
+    flops = th * (2 * C * (3 * w.dk + 2 * w.dv) + 6 * w.dk * w.dv)
+    return nbytes, flops
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel_key)
+        if not e:
+            return None
+        if e.get("source_sha") != source_sha(e.get("source", "")):
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def source_sha(rel):
+    import hashlib
+    p = os.path.join(ROOT, rel)
+    if not rel or not os.path.exists(p):
+        return None
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------------------
+# distributed plumbing (also exercised on CPU with gloo by the tests)
+# ----------------------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world > 1
+
+
+def barrier(active, device=None):
+    if active:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x, active, device):
+    """Maximum of a float over all ranks (identity on one rank)."""
+    if not active:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(tokens_per_rank, max_ms, world):
+    """Whole-job tokens/s: the units all ranks processed over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms / 1e3)
+
+
+# ----------------------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------
+
+class PrefillRunner:
+    """One prefill call per step; enough input sets are rotated that every step
+    reads inputs that are not L2-resident (sets total > 3x L2)."""
+
+    def __init__(self, w, dev, seed):
+        import gated_delta_rule_79_b200 as g
+        self.g, self.w, self.dev = g, w, dev
+        self.fn = g.kda_prefill if w.mixer == "kda" else g.gdn_prefill
+        one = device_inputs(w, dev, seed=seed)
+        set_bytes = sum(t.numel() * t.element_size() for t in one.values() if t is not None)
+        set_bytes += w.B * w.T * w.H * w.dv * 2
+        nsets = max(1, math.ceil(3 * L2_BYTES / set_bytes))
+        self.sets = [one] + [device_inputs(w, dev, seed=seed + 1 + i) for i in range(nsets - 1)]
+        self.o = [torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+                  for _ in self.sets]
+        self.s = [torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+                  for _ in self.sets]
+        self.ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev)
+        self.launches_per_step = 1
+        self.path = g.prefill_path(w.dk, w.dv, w.torch_dtype, w.mixer == "kda")
+        self.l2_note = f"{len(self.sets)} rotating input sets of {set_bytes / 2**20:.0f} MiB (> 3x L2)"
+
+    def step(self, i):
+        x = self.sets[i % len(self.sets)]
+        self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"],
+                o=self.o[i % len(self.sets)], s_final=self.s[i % len(self.sets)],
+                workspace=self.ws)
+
+
+class DecodeRunner:
+    """512 decode calls per step over a 0.5 GB state (larger than L2)."""
+
+    def __init__(self, w, dev, seed):
+        import gated_delta_rule_79_b200 as g
+        self.g, self.w, self.dev = g, w, dev
+        self.fn = g.kda_decode if w.mixer == "kda" else g.gdn_decode
+        self.x = device_inputs(w, dev, seed=seed)
+        self.state = self.x["s0"]
+        self.o = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = w.T
+        self.path = "decode (CUDA cores, fp32 state)"
+        self.l2_note = f"state of {self.state.numel() * 4 / 2**20:.0f} MiB > L2"
+
+    def step(self, i):
+        x = self.x
+        for t in range(self.w.T):
+            self.fn(x["q"][t], x["k"][t], x["v"][t], x["alpha"][t], x["beta"][t], self.state,
+                    o=self.o)
+
+
+def time_device(runner, steps, warmup, dev, active):
+    """Warm up, then time exactly `steps` steps with CUDA events on the launching
+    stream, bracketed by a barrier and a synchronize on both sides.  Also records
+    each step's own event pair (the kernel-duration evidence for the roofline)."""
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warmup):
+        runner.step(i)
+    torch.cuda.synchronize(dev)
+    barrier(active, dev)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        runner.step(warmup + i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(active, dev)
+    total_ms = t0.elapsed_time(t1)
+    per = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, per
+
+
+def time_e2e(w, dev, steps, warmup, seed):
+    """The public API with pinned host buffers: every step copies the step's
+    inputs host->device, runs the path and copies the results back."""
+    import gated_delta_rule_79_b200 as g
+    stream = torch.cuda.current_stream(dev)
+    x = device_inputs(w, dev, seed=seed + 100)
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
+    if w.decode:
+        fn = g.kda_decode if w.mixer == "kda" else g.gdn_decode
+        state = x["s0"]
+        dbuf = {k: torch.empty_like(x[k][0]) for k in ("q", "k", "v", "alpha", "beta")}
+        o = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        o_host = torch.empty((w.T, w.B, w.H, w.dv), dtype=torch.bfloat16).pin_memory()
+        h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in dbuf) * w.T
+        d2h = o_host.numel() * 2
+
+        def step():
+            for t in range(w.T):
+                for key in dbuf:
+                    dbuf[key].copy_(host[key][t], non_blocking=True)
+                fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o)
+                o_host[t].copy_(o, non_blocking=True)
+    else:
+        fn = g.kda_prefill if w.mixer == "kda" else g.gdn_prefill
+        dbuf = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
+        ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev)
+        o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        s = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        s_host = torch.empty(s.shape, dtype=s.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in dbuf.values())
+        d2h = o.numel() * 2 + s.numel() * 4
+
+        def step():
+            for key in dbuf:
+                dbuf[key].copy_(host[key], non_blocking=True)
+            fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], dbuf.get("s0"),
+               o=o, s_final=s, workspace=ws)
+            o_host.copy_(o, non_blocking=True)
+            s_host.copy_(s, non_blocking=True)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / steps
+    return {"value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ----------------------------------------------------------------------------------------
+# the oracle as CPU baseline / reference arm
+# ----------------------------------------------------------------------------------------
+
+def _oracle_slice(args):
+    """Run the oracle over one (batch, head) chain for the first `t_sample` tokens."""
+    name, b, h, t_sample = args
+    import numpy as np  # noqa: F401
+    from oracle import gated_delta_rule, decode_step
+    w = WORKLOADS[name]
+    x = slice_inputs(w.with_(T=t_sample), b, h)
+    col = lambda key: x[key][None, :, None].double().numpy()  # noqa: E731
+    s0 = None if x["s0"] is None else x["s0"][None, None].double().numpy()
+    t = time.perf_counter()
+    if w.decode:
+        st = s0
+        for i in range(t_sample):
+            _, st = decode_step(*[x[k][i][None, None].double().numpy()
+                                  for k in ("q", "k", "v", "alpha", "beta")], st)
+    else:
+        gated_delta_rule(col("q"), col("k"), col("v"), col("alpha"), col("beta"), s0)
+    return time.perf_counter() - t
+
+
+class OracleTimer:
+    """Times the oracle on the host cores over a bounded sample of workload w: a
+    spawn pool with one process per core, each running whole (batch, head) chains
+    over the first t_sample tokens, t_sample calibrated so that one timed pass
+    takes about `budget_s` seconds."""
+
+    def __init__(self, w, budget_s):
+        import multiprocessing as mp
+        self.w = w
+        self.cores = min(len(os.sched_getaffinity(0)), w.B * w.H)
+        t_cal = min(w.T, 64)
+        per_token_head = _oracle_slice((w.name, 0, 0, t_cal)) / t_cal
+        self.t_sample = max(1, min(w.T, int(budget_s / max(per_token_head, 1e-9))))
+        self.chains = [(w.name, i // w.H, i % w.H, self.t_sample) for i in range(self.cores)]
+        self.pool = mp.get_context("spawn").Pool(processes=self.cores)
+        self.pool.map(_oracle_slice, [(w.name, 0, 0, 1)] * self.cores)   # start the workers
+        self.sample = (f"{self.cores} (sequence, head) chains x {self.t_sample} tokens of "
+                       f"{w.name} per pass, fp64 numpy oracle, one spawn process per chain; "
+                       f"tokens/s = token-heads/s / H")
+
+    def rate(self):
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_slice, self.chains)
+        wall = time.perf_counter() - t0
+        return self.cores * self.t_sample / wall / self.w.H
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+# ----------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="gdn_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    w = WORKLOADS[a.workload]
+    if w.name == "gdn_seq_f32":
+        raise SystemExit("gdn_seq_f32 is a parity case, not a bench line")
+    default_steps = 5 if (w.decode or w.name == "kda_long") else 50
+    steps = a.steps if a.steps is not None else default_steps
+    warmup = max(3, a.warmup if a.warmup is not None else 5)
+    rank, world, local = dist_env()
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        ot = OracleTimer(w, budget_s=min(10.0, 150.0 / max(1, steps + warmup)))
+        for _ in range(warmup):
+            ot.rate()
+        rates = [ot.rate() for _ in range(steps)]
+        ot.close()
+        v = statistics.median(rates)
+        cores, sample = ot.cores, ot.sample
+        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": a.gpus,
+                "steps": steps, "warmup": warmup, "ms_per_step": w.B * w.T / v * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+                           "dv": w.dv, "in_dtype": w.dtype},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    active = dist_init(world, "nccl")
+    peaks, peak_kind = load_peaks()
+    runner = (DecodeRunner if w.decode else PrefillRunner)(w, dev, seed=1000 * rank)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    total_ms, per = time_device(runner, steps, warmup, dev, active)
+    clk = clocks.stop()
+    ms_step = total_ms / steps
+    max_ms = max_over_ranks(total_ms, active, dev)
+    tokens = w.B * w.T
+    value = aggregate(tokens * steps, max_ms, world)
+    nbytes, flops = algorithmic(w)
+    kern_ms = statistics.mean(per)
+    if w.decode:
+        # per-step event pairs bracket 512 launches; the kernel's own duration is
+        # that over the launches (launch gaps included, so this is conservative)
+        launch_ms = kern_ms / w.T
+        bytes_launch = nbytes / w.T
+        flops_launch = flops / w.T
+    else:
+        launch_ms, bytes_launch, flops_launch = kern_ms, nbytes, flops
+    hbm = bytes_launch / (launch_ms / 1e3) / 1e9
+    tflops = flops_launch / (launch_ms / 1e3) / 1e12
+    kernel_key = ("decode" if w.decode else f"prefill_{runner.path}") + f":{w.name}"
+    traffic = load_traffic(kernel_key)
+    roofline = {"bound": "hbm", "achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
+                "launch_ms": launch_ms}
+    extra = {}
+    if not w.decode:
+        extra["roofline_tensor"] = {
+            "bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+            "frac_of_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "algorithmic_flops_per_launch": flops_launch, "peak_source": peak_kind}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": max_ms / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if runner.path == "tensor-core" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "in_dtype": w.dtype, "out_dtype": "bf16", "chunk": 64,
+                       "kernel": runner.path, "l2": runner.l2_note,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": roofline, **extra,
+            "gpu_launches": runner.launches_per_step * steps,
+            "clocks": clk}
+    if not a.no_e2e:
+        line["e2e"] = time_e2e(w, dev, steps=max(1, min(steps, 10)), warmup=2, seed=rank)
+        if world > 1:
+            line["e2e"]["value"] *= world
+    if rank == 0 and not a.no_cpu_baseline and world == 1:
+        ot = OracleTimer(w, budget_s=12.0)
+        rate = ot.rate()
+        ot.close()
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": ot.cores,
+                                "kind": "oracle", "sample": ot.sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if active:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    del ms_step
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

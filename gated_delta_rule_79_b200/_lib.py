@@ -1,0 +1,225 @@
+"""ctypes binding of libgdr (include/gdr.h): argument marshalling only.
+
+Every function here checks tensor devices, dtypes, shapes and contiguity,
+allocates outputs with torch (device memory is torch's job), and passes raw
+pointers plus the current CUDA stream to the C ABI.  All arithmetic of the
+method runs in the library's CUDA kernels; there is no fallback.  Importing this
+module raises if libgdr.so has not been built.
+"""
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdr.so")
+
+GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = range(5)
+GDR_F32, GDR_BF16 = 0, 1
+CHUNK = 64
+
+EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
+           "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
+           "gdr_prefill_path"]
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"[gdr status {status}] {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m gated_delta_rule_79_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gdr_version.restype = i
+    lib.gdr_version.argtypes = []
+    lib.gdr_last_error.restype = ctypes.c_char_p
+    lib.gdr_last_error.argtypes = []
+    lib.gdr_prefill_workspace_bytes.restype = sz
+    lib.gdr_prefill_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    for name in ("gdn_prefill", "kda_prefill"):
+        f = getattr(lib, name)
+        f.restype = i
+        f.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    for name in ("gdn_decode", "kda_decode"):
+        f = getattr(lib, name)
+        f.restype = i
+        f.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdr_prefill_path.restype = i
+    lib.gdr_prefill_path.argtypes = [i, i, i, i]
+    lib.gdr_workspace_status.restype = i
+    lib.gdr_workspace_status.argtypes = [vp, sz, vp]
+    return lib
+
+
+lib = _load()
+
+
+def _check(status):
+    if status != GDR_OK:
+        raise GdrError(status, lib.gdr_last_error().decode())
+
+
+def _code(dtype):
+    if dtype == torch.float32:
+        return GDR_F32
+    if dtype == torch.bfloat16:
+        return GDR_BF16
+    raise TypeError(f"unsupported dtype {dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, shape, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_ws_lock = threading.Lock()
+_ws_cache = {}
+
+
+def prefill_workspace(B, T, H, dk, dv, kda, device, stream=None):
+    """Zero-initialised device workspace for a prefill call, cached per
+    (device, stream) and grown on demand.  Returns (tensor, nbytes)."""
+    need = lib.gdr_prefill_workspace_bytes(B, T, H, dk, dv, int(kda))
+    if need == 0:
+        raise GdrError(GDR_ERR_INVALID_ARG, "invalid prefill sizes")
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (device, s.cuda_stream)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < need:
+            with torch.cuda.stream(s):
+                buf = torch.zeros(max(need, 1 << 12), dtype=torch.uint8, device=device)
+            _ws_cache[key] = buf
+    return buf, buf.numel()
+
+
+def _prefill(kda, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream, workspace):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, d_k]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    dt = q.dtype
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(alpha, "alpha", (B, T, H, dk) if kda else (B, T, H), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if s0 is not None:
+        _need(s0, "s0", (B, H, dv, dk), torch.float32, dev)
+    out_dtype = out_dtype or dt
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev)
+    _need(o, "o", (B, T, H, dv), out_dtype, dev)
+    if s_final is None:
+        s_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    elif s_final is not False:
+        _need(s_final, "s_final", (B, H, dv, dk), torch.float32, dev)
+    sf = None if s_final is False else s_final
+    if workspace is None:
+        ws, nws = prefill_workspace(B, T, H, dk, dv, kda, dev, stream)
+    else:
+        ws, nws = workspace, workspace.numel() * workspace.element_size()
+    fn = lib.kda_prefill if kda else lib.gdn_prefill
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(s0), _ptr(o), _ptr(sf),
+              B, T, H, dk, dv, _code(dt), _code(out_dtype), chunk, _ptr(ws), nws,
+              _stream(dev, stream)))
+    return o, sf
+
+
+def gdn_prefill(q, k, v, alpha, beta, s0=None, *, out_dtype=None, o=None, s_final=None,
+                chunk=CHUNK, stream=None, workspace=None):
+    """Gated DeltaNet chunked prefill (scalar gate alpha [B, T, H]).
+
+    q, k [B, T, H, d_k] and v [B, T, H, d_v] in float32 or bfloat16; alpha, beta
+    float32; s0 [B, H, d_v, d_k] float32 or None.  Returns (o, s_final); pass
+    s_final=False to skip writing the final state, or s_final=s0 to carry in place.
+    """
+    return _prefill(False, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream,
+                    workspace)
+
+
+def kda_prefill(q, k, v, alpha, beta, s0=None, *, out_dtype=None, o=None, s_final=None,
+                chunk=CHUNK, stream=None, workspace=None):
+    """Kimi Delta Attention chunked prefill (per-channel gate alpha [B, T, H, d_k]);
+    otherwise as ``gdn_prefill``."""
+    return _prefill(True, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream,
+                    workspace)
+
+
+def _decode(kda, q, k, v, alpha, beta, state, out_dtype, o, stream):
+    if q.dim() != 3:
+        raise ValueError("q must be [N, H, d_k]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    dt = q.dtype
+    _need(q, "q", (N, H, dk), dt, dev)
+    _need(k, "k", (N, H, dk), dt, dev)
+    _need(v, "v", (N, H, dv), dt, dev)
+    _need(alpha, "alpha", (N, H, dk) if kda else (N, H), torch.float32, dev)
+    _need(beta, "beta", (N, H), torch.float32, dev)
+    _need(state, "state", (N, H, dv, dk), torch.float32, dev)
+    out_dtype = out_dtype or dt
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=out_dtype, device=dev)
+    _need(o, "o", (N, H, dv), out_dtype, dev)
+    fn = lib.kda_decode if kda else lib.gdn_decode
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(o),
+              N, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream)))
+    return o
+
+
+def gdn_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
+    """One Gated DeltaNet decode step for N sequences; ``state`` [N, H, d_v, d_k]
+    float32 is updated in place.  Returns o [N, H, d_v]."""
+    return _decode(False, q, k, v, alpha, beta, state, out_dtype, o, stream)
+
+
+def kda_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
+    """One Kimi Delta Attention decode step (alpha [N, H, d_k]); as ``gdn_decode``."""
+    return _decode(True, q, k, v, alpha, beta, state, out_dtype, o, stream)
+
+
+def prefill_path(dk, dv, dtype, kda):
+    """"tensor-core" or "cuda-core": which prefill kernel serves these parameters."""
+    p = lib.gdr_prefill_path(dk, dv, _code(dtype), int(kda))
+    if p < 0:
+        raise GdrError(GDR_ERR_UNSUPPORTED, f"no prefill kernel for d_k={dk} d_v={dv}")
+    return "tensor-core" if p == 1 else "cuda-core"
+
+
+def workspace_status(workspace, stream=None):
+    """Synchronise and read/clear the device status word of a prefill workspace;
+    raises GdrError(GDR_ERR_TIMEOUT) if a bounded device wait gave up."""
+    dev = workspace.device
+    _check(lib.gdr_workspace_status(_ptr(workspace), workspace.numel(), _stream(dev, stream)))

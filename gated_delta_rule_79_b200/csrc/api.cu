@@ -1,0 +1,191 @@
+// C ABI of libgdr (declared in include/gdr.h): argument validation, kernel
+// selection and error reporting.  Every entry point validates all of its
+// arguments on the host before anything is enqueued, so a rejected call leaves
+// the device untouched.
+
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "gdr.h"
+#include "launch.h"
+
+namespace gdr {
+
+static thread_local std::string g_last_error;
+
+static gdr_status fail(gdr_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+static gdr_status ok() {
+  g_last_error.clear();
+  return GDR_OK;
+}
+
+static bool head_ok(int d) { return d == 32 || d == 64 || d == 128; }
+static bool dtype_ok(int t) { return t == GDR_F32 || t == GDR_BF16; }
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Bytes of the status word area at the start of a prefill workspace.
+constexpr size_t kStatusBytes = 256;
+
+bool tc_prefill_supported(const PrefillArgs& a);   // prefill_tc.cu
+size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+
+static gdr_status prefill(bool kda, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, const float* s0, void* o,
+                          float* s_final, int B, int T, int H, int dk, int dv, int in_dtype,
+                          int out_dtype, int chunk, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  const char* fn = kda ? "kda_prefill" : "gdn_prefill";
+  if (B < 0 || T < 0 || H < 0)
+    return fail(GDR_ERR_INVALID_ARG, "%s: negative size B=%d T=%d H=%d", fn, B, T, H);
+  if (!head_ok(dk) || !head_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "%s: d_k=%d d_v=%d (supported: 32, 64, 128)", fn, dk, dv);
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype))
+    return fail(GDR_ERR_INVALID_ARG, "%s: bad dtype in=%d out=%d", fn, in_dtype, out_dtype);
+  if (chunk != GDR_CHUNK)
+    return fail(GDR_ERR_UNSUPPORTED, "%s: chunk=%d (only %d is supported)", fn, chunk, GDR_CHUNK);
+  const size_t need = gdr_prefill_workspace_bytes(B, T, H, dk, dv, kda);
+  if (need == 0) return fail(GDR_ERR_INVALID_ARG, "%s: sizes overflow", fn);
+  if (!workspace || ws_bytes < need)
+    return fail(GDR_ERR_INVALID_ARG, "%s: workspace %p of %zu bytes, need %zu", fn, workspace,
+                ws_bytes, need);
+  if (((uintptr_t)workspace & 255u) != 0)
+    return fail(GDR_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t state_bytes = (size_t)B * H * dv * dk * sizeof(float);
+  if (B == 0 || H == 0) return ok();
+  if (T == 0) {
+    if (!s_final) return ok();
+    if (!aligned16(s_final)) return fail(GDR_ERR_INVALID_ARG, "%s: s_final misaligned", fn);
+    cudaError_t e = s0 ? (s0 == s_final ? cudaSuccess
+                                        : cudaMemcpyAsync(s_final, s0, state_bytes,
+                                                          cudaMemcpyDeviceToDevice, st))
+                       : cudaMemsetAsync(s_final, 0, state_bytes, st);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    return ok();
+  }
+  const void* need_ptrs[] = {q, k, v, alpha, beta, o};
+  const char* names[] = {"q", "k", "v", "alpha", "beta", "o"};
+  for (int i = 0; i < 6; ++i) {
+    if (!need_ptrs[i]) return fail(GDR_ERR_INVALID_ARG, "%s: %s is NULL", fn, names[i]);
+    if (!aligned16(need_ptrs[i]))
+      return fail(GDR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
+  }
+  if ((s0 && !aligned16(s0)) || (s_final && !aligned16(s_final)))
+    return fail(GDR_ERR_INVALID_ARG, "%s: s0/s_final not 16-byte aligned", fn);
+  PrefillArgs a{q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv,
+                in_dtype, out_dtype, kda, workspace, ws_bytes};
+  cudaError_t e = tc_prefill_supported(a) ? launch_prefill_tc(a, st) : launch_prefill_simt(a, st);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return ok();
+}
+
+static gdr_status decode(bool kda, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* beta, float* state, void* o, int N,
+                         int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
+  const char* fn = kda ? "kda_decode" : "gdn_decode";
+  if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "%s: negative size N=%d H=%d", fn, N, H);
+  if (!head_ok(dk) || !head_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "%s: d_k=%d d_v=%d (supported: 32, 64, 128)", fn, dk, dv);
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype))
+    return fail(GDR_ERR_INVALID_ARG, "%s: bad dtype in=%d out=%d", fn, in_dtype, out_dtype);
+  if ((long long)N * H > (1LL << 31) / 4)
+    return fail(GDR_ERR_INVALID_ARG, "%s: N*H too large", fn);
+  if (N == 0 || H == 0) return ok();
+  const void* need_ptrs[] = {q, k, v, alpha, beta, state, o};
+  const char* names[] = {"q", "k", "v", "alpha", "beta", "state", "o"};
+  for (int i = 0; i < 7; ++i) {
+    if (!need_ptrs[i]) return fail(GDR_ERR_INVALID_ARG, "%s: %s is NULL", fn, names[i]);
+    if (!aligned16(need_ptrs[i]))
+      return fail(GDR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
+  }
+  DecodeArgs a{q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype, kda};
+  cudaError_t e = launch_decode(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace gdr
+
+extern "C" {
+
+int gdr_version(void) { return 100; }
+
+const char* gdr_last_error(void) { return gdr::g_last_error.c_str(); }
+
+size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, int kda) {
+  if (B < 0 || T < 0 || H < 0) return 0;
+  if ((long long)B * H > (1LL << 24) || T > (1 << 28)) return 0;
+  return gdr::kStatusBytes + gdr::tc_prefill_workspace(B, T, H, dk, dv, kda != 0);
+}
+
+gdr_status gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const float* s0, void* o, float* s_final, int B,
+                       int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  return gdr::prefill(false, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
+                      out_dtype, chunk, workspace, ws_bytes, stream);
+}
+
+gdr_status kda_prefill(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const float* s0, void* o, float* s_final, int B,
+                       int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  return gdr::prefill(true, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
+                      out_dtype, chunk, workspace, ws_bytes, stream);
+}
+
+gdr_status gdn_decode(const void* q, const void* k, const void* v, const float* alpha,
+                      const float* beta, float* state, void* o, int N, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream) {
+  return gdr::decode(false, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
+                     stream);
+}
+
+gdr_status kda_decode(const void* q, const void* k, const void* v, const float* alpha,
+                      const float* beta, float* state, void* o, int N, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream) {
+  return gdr::decode(true, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
+                     stream);
+}
+
+int gdr_prefill_path(int dk, int dv, int in_dtype, int kda) {
+  if (!gdr::head_ok(dk) || !gdr::head_ok(dv) || !gdr::dtype_ok(in_dtype)) return -1;
+  gdr::PrefillArgs a{};
+  a.dk = dk;
+  a.dv = dv;
+  a.in_dtype = in_dtype;
+  a.kda = kda != 0;
+  return gdr::tc_prefill_supported(a) ? 1 : 0;
+}
+
+gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || ws_bytes < gdr::kStatusBytes)
+    return gdr::fail(GDR_ERR_INVALID_ARG, "gdr_workspace_status: bad workspace");
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && word != 0) e = cudaMemsetAsync(workspace, 0, sizeof word, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess)
+    return gdr::fail(GDR_ERR_CUDA, "gdr_workspace_status: %s", cudaGetErrorString(e));
+  if (word != 0)
+    return gdr::fail(GDR_ERR_TIMEOUT, "a bounded device wait gave up (status word 0x%08x)", word);
+  return gdr::ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// Internal launcher declarations of libgdr (host side).  The C ABI in gdr.h
+// validates arguments and then calls these.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdr {
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  const float* beta;
+  const float* s0;      // may be null (zeros)
+  void* o;
+  float* s_final;       // may be null
+  int B, T, H, dk, dv;
+  int in_dtype, out_dtype;
+  bool kda;
+  void* workspace;
+  size_t ws_bytes;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  const float* beta;
+  float* state;
+  void* o;
+  int N, H, dk, dv;
+  int in_dtype, out_dtype;
+  bool kda;
+};
+
+// Each returns cudaSuccess or the launch error; messages are set by the caller.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
+
+}  // namespace gdr

@@ -1,0 +1,153 @@
+/*
+ * gdr.h - C ABI of libgdr: the gated delta rule token mixers (GDN and KDA) on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation.  "Super Apriel: One Checkpoint, Many Speeds", §2A (Mixer
+ * Vocabulary) names two recurrent mixers: Gated DeltaNet (GDN), the delta rule
+ * with a scalar gate, and Kimi Delta Attention (KDA), the delta rule with a
+ * channel-wise gate; §1 and §4 (context-length scaling) rest on their state
+ * having a fixed size.  For every (sequence, head) the state S is a d_v x d_k
+ * fp32 matrix and each token t applies
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * with alpha_t one scalar per (token, head) for GDN and one value per key
+ * channel (a d_k-vector) for KDA.  No scaling is applied to q; callers that want
+ * 1/sqrt(d_k) or L2-normalised q/k apply it before the call.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, dense
+ *     (row-major, no strides), and 16-byte aligned.  The library never frees or
+ *     retains them after the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  A GDR_OK return means the arguments
+ *     were accepted and the kernels were enqueued; device-side problems surface
+ *     at the caller's next synchronisation (or through gdr_workspace_status).
+ *   - Nothing throws across the ABI.  On a non-OK status nothing was enqueued,
+ *     and gdr_last_error() returns a message for the calling thread.
+ *   - alpha is taken as the gate itself, in [0, 1]; the kernels work with
+ *     max(log(alpha), -GDR_LOG_GATE_FLOOR), so a gate below e^-30 acts as e^-30
+ *     (a factor below 1e-13 on what the state carried).  Values are not checked
+ *     on the device.
+ *   - Supported head sizes: d_k, d_v in {32, 64, 128}.  The chunk length of the
+ *     prefill is 64 tokens; the last chunk of a sequence may be shorter.
+ *   - The library is thread-safe for calls on different streams; calls that
+ *     share a workspace must not overlap on the device.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdr_status {
+  GDR_OK = 0,
+  GDR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad enum    */
+  GDR_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for     */
+  GDR_ERR_CUDA = 3,          /* a CUDA runtime call failed (message says which) */
+  GDR_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up             */
+} gdr_status;
+
+typedef enum gdr_dtype {
+  GDR_F32 = 0,               /* IEEE fp32                                      */
+  GDR_BF16 = 1               /* bfloat16                                       */
+} gdr_dtype;
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#define GDR_CHUNK 64
+#define GDR_LOG_GATE_FLOOR 30.0f
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+GDR_API int gdr_version(void);
+
+/* Message describing the last non-OK status returned on the calling thread
+ * (empty string if none).  The pointer stays valid until the thread's next call
+ * into the library. */
+GDR_API const char* gdr_last_error(void);
+
+/* Bytes of device workspace that gdn_prefill / kda_prefill need for these
+ * sizes (kda != 0 selects KDA).  The workspace holds the device status word of
+ * the bounded waits and the per-chunk exchange area of the prefill kernels.  It
+ * must be zero-filled once when allocated; the library leaves it ready for the
+ * next call.  Returns 0 when the sizes are invalid. */
+GDR_API size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, int kda);
+
+/* Chunked prefill: runs the recurrence over T tokens for B sequences and H heads
+ * and returns every output plus the final state.
+ *
+ *   q, k     [B, T, H, d_k]   in_dtype
+ *   v        [B, T, H, d_v]   in_dtype
+ *   alpha    GDN: [B, T, H] fp32, one gate per (token, head)
+ *            KDA: [B, T, H, d_k] fp32, one gate per key channel
+ *   beta     [B, T, H] fp32
+ *   s0       [B, H, d_v, d_k] fp32 initial state, or NULL for zeros
+ *   o        [B, T, H, d_v]   out_dtype (written)
+ *   s_final  [B, H, d_v, d_k] fp32 (written), or NULL to skip; may be the same
+ *            pointer as s0 (in-place carry), must not otherwise overlap inputs
+ *   chunk    must be GDR_CHUNK (64)
+ *   workspace, ws_bytes: at least gdr_prefill_workspace_bytes(...) bytes,
+ *            zero-filled at allocation, 256-byte aligned
+ * B, T or H equal to 0 is a valid empty call (with T == 0, s_final receives s0,
+ * or zeros when s0 is NULL).  in_dtype GDR_F32 runs the fp32 CUDA-core kernel;
+ * GDR_BF16 runs the tensor-core kernel where one exists for (d_k, d_v). */
+GDR_API gdr_status gdn_prefill(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const float* s0,
+                       void* o, float* s_final,
+                       int B, int T, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Same contract as gdn_prefill with the per-channel gate alpha [B, T, H, d_k]. */
+GDR_API gdr_status kda_prefill(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const float* s0,
+                       void* o, float* s_final,
+                       int B, int T, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* One decode step: one new token for each of N sequences, the state updated IN
+ * PLACE.
+ *
+ *   q, k     [N, H, d_k]   in_dtype
+ *   v        [N, H, d_v]   in_dtype
+ *   alpha    GDN: [N, H] fp32; KDA: [N, H, d_k] fp32
+ *   beta     [N, H] fp32
+ *   state    [N, H, d_v, d_k] fp32, read and overwritten with S_t
+ *   o        [N, H, d_v]   out_dtype (written), o = S_t q_t
+ * N or H equal to 0 is a valid empty call.  No workspace is used. */
+GDR_API gdr_status gdn_decode(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, void* o,
+                      int N, int H, int dk, int dv, int in_dtype, int out_dtype,
+                      void* stream);
+
+/* Same contract as gdn_decode with the per-channel gate alpha [N, H, d_k]. */
+GDR_API gdr_status kda_decode(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, void* o,
+                      int N, int H, int dk, int dv, int in_dtype, int out_dtype,
+                      void* stream);
+
+/* Which prefill kernel a call with these parameters runs: 1 = the bf16
+ * tensor-core (tcgen05) kernel, 0 = the fp32 CUDA-core kernel, -1 = the
+ * parameters are not supported.  Pure host query, no CUDA call. */
+GDR_API int gdr_prefill_path(int dk, int dv, int in_dtype, int kda);
+
+/* Synchronises `stream`, reads the device status word in `workspace` and clears
+ * it.  Returns GDR_OK, GDR_ERR_TIMEOUT if a bounded device-side wait of a
+ * prefill kernel gave up since the last check (the outputs of that call are
+ * then undefined), or GDR_ERR_CUDA. */
+GDR_API gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* GDR_H_ */

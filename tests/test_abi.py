@@ -1,0 +1,97 @@
+"""The C-ABI library: it loads, exports every symbol include/gdr.h declares, and
+rejects bad arguments on the host (these calls return before any CUDA work, so
+they run without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"GDR_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+@pytest.fixture(scope="module")
+def g():
+    import gated_delta_rule_79_b200 as pkg
+    return pkg
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_symbols()
+    for required in ("gdn_prefill", "kda_prefill", "gdn_decode", "kda_decode",
+                     "gdr_prefill_workspace_bytes", "gdr_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(g):
+    lib = ctypes.CDLL(g.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(_declared_symbols()) <= set(g.EXPORTS) | {"gdr_version"}
+
+
+def test_version_and_workspace(g):
+    assert g.lib.gdr_version() >= 100
+    n = g.lib.gdr_prefill_workspace_bytes(1, 4096, 32, 128, 128, 0)
+    assert n >= 256
+    assert g.lib.gdr_prefill_workspace_bytes(-1, 1, 1, 128, 128, 0) == 0
+
+
+def _prefill(g, fn, **kw):
+    a = dict(q=1 << 20, k=1 << 20, v=1 << 20, alpha=1 << 20, beta=1 << 20, s0=None, o=1 << 20,
+             s_final=None, B=1, T=8, H=1, dk=64, dv=64, i=1, oo=1, chunk=64, ws=1 << 20,
+             nws=4096, stream=None)
+    a.update(kw)
+    f = getattr(g.lib, fn)
+    return f(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["s0"], a["o"], a["s_final"],
+             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["i"], a["oo"], a["chunk"], a["ws"],
+             a["nws"], a["stream"])
+
+
+@pytest.mark.parametrize("fn", ["gdn_prefill", "kda_prefill"])
+def test_prefill_rejects_bad_arguments(g, fn):
+    assert _prefill(g, fn, dk=48) == g.GDR_ERR_UNSUPPORTED
+    assert "d_k=48" in g.lib.gdr_last_error().decode()
+    assert _prefill(g, fn, dv=256) == g.GDR_ERR_UNSUPPORTED
+    assert _prefill(g, fn, chunk=32) == g.GDR_ERR_UNSUPPORTED
+    assert _prefill(g, fn, B=-1) == g.GDR_ERR_INVALID_ARG
+    assert _prefill(g, fn, i=7) == g.GDR_ERR_INVALID_ARG
+    assert _prefill(g, fn, ws=None) == g.GDR_ERR_INVALID_ARG
+    assert _prefill(g, fn, nws=16) == g.GDR_ERR_INVALID_ARG
+    assert _prefill(g, fn, ws=(1 << 20) + 16) == g.GDR_ERR_INVALID_ARG   # not 256-aligned
+    assert _prefill(g, fn, q=None) == g.GDR_ERR_INVALID_ARG
+    assert "q is NULL" in g.lib.gdr_last_error().decode()
+    assert _prefill(g, fn, v=(1 << 20) + 8) == g.GDR_ERR_INVALID_ARG     # misaligned
+    # empty batches are valid and enqueue nothing
+    assert _prefill(g, fn, B=0) == g.GDR_OK
+    assert _prefill(g, fn, H=0) == g.GDR_OK
+    assert g.lib.gdr_last_error().decode() == ""
+
+
+@pytest.mark.parametrize("fn", ["gdn_decode", "kda_decode"])
+def test_decode_rejects_bad_arguments(g, fn):
+    f = getattr(g.lib, fn)
+    P = 1 << 20
+
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, alpha=P, beta=P, state=P, o=P, N=4, H=2, dk=128, dv=128,
+                 i=1, oo=1)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["state"], a["o"], a["N"],
+                 a["H"], a["dk"], a["dv"], a["i"], a["oo"], None)
+    assert call(dk=16) == g.GDR_ERR_UNSUPPORTED
+    assert call(N=-2) == g.GDR_ERR_INVALID_ARG
+    assert call(state=None) == g.GDR_ERR_INVALID_ARG
+    assert call(alpha=P + 4) == g.GDR_ERR_INVALID_ARG
+    assert call(oo=3) == g.GDR_ERR_INVALID_ARG
+    assert call(N=0) == g.GDR_OK
