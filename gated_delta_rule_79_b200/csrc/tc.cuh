@@ -1,13 +1,13 @@
 // sm_100a tensor-core plumbing: tcgen05 MMA issue, TMEM allocation and access,
 // shared-memory matrix descriptors, mbarriers with bounded waits.
 //
-// Operand tiles live in shared memory in the 128-byte-swizzled layout: a tile
-// of R rows (R a multiple of 8) by 32*NP fp32 columns is stored as NP column
-// panels of R rows x 128 bytes; inside a panel the 16-byte chunk j of row r sits
-// at chunk position j ^ (r % 8).  The same physical tile serves as a K-major
-// operand (the row index is M or N, the column index is K) or as an MN-major
-// operand (the row index is K, the column index is M or N); only the
-// descriptor differs.  Tile bases are 1024-byte aligned.
+// Operand tiles live in shared memory in the 128-byte-swizzled K-major layout: a
+// tile of R rows (R a multiple of 8; the row index is M or N) by 32*NP fp32
+// columns (the K index) is stored as NP column panels of R rows x 128 bytes;
+// inside a panel the 16-byte chunk j of row r sits at chunk position j ^ (r % 8).
+// Tile bases are 1024-byte aligned.  (MN-major tf32 operands would need the
+// different 32-byte-granular swizzle, so products that want the other
+// orientation use a transposed K-major copy instead.)
 #pragma once
 
 #include <stdint.h>
@@ -149,11 +149,29 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- TMA --------------------------------------------------------------------------------
+
+// 4-D tiled bulk tensor load global -> shared, completing `bytes` on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
+                                            int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+         "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---- mbarrier --------------------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count)
                : "memory");
+}
+// Arrive once and add `bytes` to the transaction count the current phase waits for.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
