@@ -1,0 +1,71 @@
+"""bench.py's host-side logic: algorithmic work counts, and the multi-rank timing
+plumbing (barrier, max over ranks, whole-job aggregation) on CPU with gloo,
+world_size 2."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from synth import WORKLOADS
+
+
+def test_algorithmic_counts():
+    nb, fl = bench.algorithmic(WORKLOADS["gdn_prefill"])
+    th = 4096 * 32
+    assert fl == th * 180224
+    assert nb == th * 1032 + 32 * 128 * 128 * 4           # + final state write
+    nb, _ = bench.algorithmic(WORKLOADS["kda_prefill"])
+    assert nb == th * 1540 + 32 * 128 * 128 * 4
+    nb, _ = bench.algorithmic(WORKLOADS["decode_gdn"])
+    assert nb == 2 * 256 * 32 * 128 * 128 * 4 * 512        # state read + write per step
+    nb, _ = bench.algorithmic(WORKLOADS["kda_long"])
+    assert nb == 4 * 65536 * 32 * 1540 + 2 * 4 * 32 * 128 * 128 * 4
+
+
+def test_aggregate_single_rank():
+    assert bench.aggregate(1000, 500.0, 1) == pytest.approx(2000.0)
+    assert bench.max_over_ranks(3.5, False, torch.device("cpu")) == 3.5
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, _ = bench.dist_env()
+    active = bench.dist_init(w, "gloo")
+    bench.barrier(active, torch.device("cpu"))
+    my_ms = 100.0 + 50.0 * r                       # rank 1 is the slow one
+    mx = bench.max_over_ranks(my_ms, active, torch.device("cpu"))
+    value = bench.aggregate(tokens_per_rank=4096, max_ms=mx, world=w)
+    bench.barrier(active, torch.device("cpu"))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, active, mx, value))
+
+
+def test_two_rank_gloo_max_and_aggregate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for r, active, mx, value in res:
+        assert active
+        assert mx == 150.0                          # max over ranks, not the local time
+        assert value == pytest.approx(4096 * 2 / 0.150)
