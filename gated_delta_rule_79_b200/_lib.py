@@ -22,7 +22,7 @@ CHUNK = 64
 
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
-           "gdr_prefill_path"]
+           "gdr_prefill_path", "gdn_prefill_noalloc"]
 
 
 class GdrError(RuntimeError):
@@ -52,6 +52,8 @@ def _load():
         f = getattr(lib, name)
         f.restype = i
         f.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    lib.gdn_prefill_noalloc.restype = i
+    lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdr_prefill_path.restype = i
     lib.gdr_prefill_path.argtypes = [i, i, i, i]
     lib.gdr_workspace_status.restype = i

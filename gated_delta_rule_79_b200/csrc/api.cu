@@ -27,6 +27,8 @@ static gdr_status fail(gdr_status s, const char* fmt, ...) {
   return s;
 }
 
+int report_error(int s, const char* msg) { return fail((gdr_status)s, "%s", msg); }
+
 static gdr_status ok() {
   g_last_error.clear();
   return GDR_OK;

@@ -36,6 +36,9 @@ struct DecodeArgs {
   bool kda;
 };
 
+// Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
+int report_error(int s, const char* msg);
+
 // Each returns cudaSuccess or the launch error; messages are set by the caller.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);

@@ -135,6 +135,26 @@ GDR_API gdr_status kda_decode(const void* q, const void* k, const void* v,
                       int N, int H, int dk, int dv, int in_dtype, int out_dtype,
                       void* stream);
 
+/* gdn_prefill for callers that cannot allocate device memory.  The paper has no
+ * counterpart to this entry point; it exists for callers such as serving loops
+ * that must never stall the device (cudaMalloc and cudaFree can synchronize it)
+ * and embedders whose device memory is owned by another allocator under a fixed
+ * budget.  Arguments, results and errors are those of gdn_prefill without the
+ * workspace: the library uses a static device array of 4096 bytes instead,
+ * reserved on every GPU that loads the library until the process exits.  Sizes
+ * that would need more scratch are rejected with GDR_ERR_INVALID_ARG.  The
+ * first call on a device looks up the array's device address with the device
+ * current, so make that first call before any stream capture.  The call
+ * allocates nothing and clears the array's status word after launching, so
+ * device-side timeouts of this variant are not reported (use gdn_prefill with a
+ * workspace and gdr_workspace_status for that).  All calls share the one array:
+ * calls that overlap on the GPU (streams without ordering between them) race. */
+GDR_API gdr_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const float* s0,
+                       void* o, float* s_final,
+                       int B, int T, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk, void* stream);
+
 /* Which prefill kernel a call with these parameters runs: 1 = the bf16
  * tensor-core (tcgen05) kernel, 0 = the fp32 CUDA-core kernel, -1 = the
  * parameters are not supported.  Pure host query, no CUDA call. */
