@@ -242,7 +242,7 @@ class DecodeRunner:
                     o=self.o)
 
 
-def time_device(runner, steps, warmup, dev, active):
+def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
     """Warm up, then time exactly `steps` steps with CUDA events on the launching
     stream, bracketed by a barrier and a synchronize on both sides.  Also records
     each step's own event pair (the kernel-duration evidence for the roofline)."""
@@ -250,6 +250,14 @@ def time_device(runner, steps, warmup, dev, active):
     for i in range(warmup):
         runner.step(i)
     torch.cuda.synchronize(dev)
+    # Soak: keep running the same steps (untimed) for about half a second so that
+    # the clock sampler sees the GPU under this load right before the timed region.
+    t_end = time.perf_counter() + soak_s
+    i = warmup
+    while time.perf_counter() < t_end:
+        runner.step(i)
+        i += 1
+        torch.cuda.synchronize(dev)
     barrier(active, dev)
     torch.cuda.synchronize(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -469,6 +477,7 @@ def main():
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "in_dtype": w.dtype, "out_dtype": "bf16", "chunk": 64,
                        "kernel": runner.path, "l2": runner.l2_note,
+                       "clocks_window": "0.5 s soak of the same steps, then the timed region",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roofline, **extra,
             "gpu_launches": runner.launches_per_step * steps,

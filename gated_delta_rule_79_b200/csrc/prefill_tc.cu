@@ -19,7 +19,7 @@
 // rounding of the computed operands (T, U, P, the state) costs about 3e-3
 // normwise error, more than the 2e-3 budget; tf32 costs about 4e-4.
 //
-// Work split: one CTA (128 threads) per (batch, head, 32-wide slice of d_v) walks
+// Work split: one CTA (256 threads) per (batch, head, 32-wide slice of d_v) walks
 // the chunks in order; the TMA load of chunk c+1 overlaps the work on chunk c.
 // The state slice S^T (128 x 32 fp32) lives in tensor memory as an accumulator
 // and in registers (thread c owns row c); a tf32 copy S_s in shared memory is
@@ -46,15 +46,15 @@ using namespace tc;
 constexpr int kC = GDR_CHUNK;
 constexpr int kDK = 128;
 constexpr int kDVS = 32;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr int OFF_QK = 0;                  // fp32 [128][128]: rows 0-63 q, 64-127 k    64 KB
 constexpr int OFF_KT = OFF_QK + 65536;     // fp32 [128 c][64 j]  k transposed          32 KB
 constexpr int OFF_P = OFF_KT + 32768;      // fp32 [64 t][64 j]                         16 KB
 constexpr int OFF_TM = OFF_P + 16384;      // fp32 T [64][64]; X scratch in the solve   16 KB
-constexpr int OFF_RT = OFF_TM + 16384;     // fp32 [32 v][64 j]; A scratch (16 KB) in prep
-constexpr int OFF_UT = OFF_RT + 8192;      // fp32 [32 v][64 j]
+constexpr int OFF_RT = OFF_TM + 16384;     // fp32 [32 v][64 j]; A scratch (16 KB over RT+UT)
+constexpr int OFF_UT = OFF_RT + 8192;      //   in prep; P U exchange [64][32] at the end
 constexpr int OFF_UPT = OFF_UT + 8192;     // fp32 [32 v][64 j]; Z scratch in the solve
 constexpr int OFF_SS = OFF_UPT + 8192;     // fp32 [32 v][128 c]  state operand          16 KB
 constexpr int OFF_VF = OFF_SS + 16384;     // fp32 [64 j][32 v]   v slice                 8 KB
@@ -66,12 +66,11 @@ constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // tensor-memory columns
-constexpr uint32_t TM_G = 0;     // Gram, M=128 x 64
-constexpr uint32_t TM_U = 64;    // U, M=64 x 32
-constexpr uint32_t TM_Y = 96;    // K S0^T, M=64 x 32
-constexpr uint32_t TM_O1 = 128;  // Q S0^T, M=64 x 32
-constexpr uint32_t TM_O2 = 160;  // P U, M=64 x 32
-constexpr uint32_t TM_S = 192;   // S^T, M=128 x 32
+constexpr uint32_t TM_G = 0;     // Gram [q; k] k^T, M=128 x 64
+constexpr uint32_t TM_OY = 64;   // [q; k] S0^T, M=128 x 32: rows 0-63 O1, rows 64-127 Y
+constexpr uint32_t TM_U = 96;    // U, M=64 x 32
+constexpr uint32_t TM_O2 = 128;  // P U, M=64 x 32
+constexpr uint32_t TM_S = 160;   // S^T, M=128 x 32
 constexpr uint32_t TM_COLS = 256;
 
 constexpr uint32_t kDrainLimit = 1u << 26;
@@ -123,6 +122,17 @@ __device__ __forceinline__ void bf16x8(const unsigned char* p, float4& a, float4
 // row and a column of 32 consecutive entries fall in distinct banks.
 __device__ __forceinline__ int sx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
 
+// Four consecutive entries (row k, columns c4 .. c4+3, c4 a multiple of 4) of an sx()
+// tile with one 16-byte load: the XOR by the row keeps aligned groups of four
+// together and permutes inside a group by (k & 3), which klo must equal (callers pass
+// an unrolled loop index, so the selection folds away at compile time).
+__device__ __forceinline__ void ld4_sx(const float* base, int k, int klo, int c4, float (&e)[4]) {
+  const float4 f = *reinterpret_cast<const float4*>(base + k * 64 + (c4 ^ (k & 28)));
+  const float v[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+  for (int x = 0; x < 4; ++x) e[x] = v[x ^ klo];
+}
+
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -147,11 +157,14 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   float* Xs = reinterpret_cast<float*>(tTM);     // solve scratch, sx() layout
   float* As = reinterpret_cast<float*>(tRT);     // 16 KB over RT + UT, sx() layout
   float* Zs = reinterpret_cast<float*>(tUPT);    // [3][16][16]
+  float* Ox = reinterpret_cast<float*>(tRT);     // P U exchange [64 t][32 v], row-XOR layout
   SmallSmem& ss = *reinterpret_cast<SmallSmem*>(sm + OFF_SMALL);
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ss.mma_bar);
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(&ss.tma_bar);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3;          // TMEM lane quarter this warp may access
+  const int hw = warp >> 2;         // which half of the CTA (splits columns)
   const int nslice = dv / kDVS;
   const int slice = blockIdx.x % nslice;
   const int bh = blockIdx.x / nslice;
@@ -170,7 +183,7 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = ss.tmem;
-  const uint32_t tlane = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lane quarter
+  const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
   uint32_t mphase = 0, tphase = 0;
   bool tma_inflight = false;
 
@@ -208,18 +221,19 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t aQK = smem_u32(tQK), aKT = smem_u32(tKT), aP = smem_u32(tP), aTM = smem_u32(tTM);
   const uint32_t aRT = smem_u32(tRT), aUT = smem_u32(tUT), aUPT = smem_u32(tUPT);
   const uint32_t aSS = smem_u32(tSS);
-  const uint64_t dQ = sdesc(aQK, 16, 1024), dK = sdesc(aQK + 64 * 128, 16, 1024);
+  const uint64_t dQK = sdesc(aQK, 16, 1024), dK = sdesc(aQK + 64 * 128, 16, 1024);
   const uint64_t dKT = sdesc(aKT, 16, 1024), dP = sdesc(aP, 16, 1024), dTM = sdesc(aTM, 16, 1024);
   const uint64_t dRT = sdesc(aRT, 16, 1024), dUT = sdesc(aUT, 16, 1024);
   const uint64_t dUPT = sdesc(aUPT, 16, 1024), dSS = sdesc(aSS, 16, 1024);
 
-  // ---- initial state: thread c holds S0[v0 + v][c]; S_s gets a tf32 copy --------------
+  // ---- initial state: thread c < 128 holds S0[v0 + v][c]; S_s gets a tf32 copy ---------
   const long sbase = ((long)b * H + h) * (long)dv * kDK;
   float st[kDVS];
+  if (tid < kDK) {
 #pragma unroll
-  for (int vv = 0; vv < kDVS; ++vv) {
-    st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
-    st_tile(tSS, kDVS, vv, tid, st[vv]);
+    for (int vv = 0; vv < kDVS; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
+#pragma unroll
+    for (int vv = 0; vv < kDVS; ++vv) st_tile(tSS, kDVS, vv, tid, st[vv]);
   }
 
   bool aborted = false;
@@ -234,39 +248,39 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       ss.g[tid] = log_gate_accurate(a_next);
       ss.beta[tid] = b_next;
     }
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      const int i = tid + kThreads * n;          // 1024 groups of 8 bf16 per tensor
-      const int t = i >> 4, q8 = i & 15;
-      float4 x0, x1;
-      bf16x8(stg + STG_Q + t * 256 + q8 * 16, x0, x1);
-      *reinterpret_cast<float4*>(tQK + swz_off4(t, 2 * q8, 128)) = x0;
-      *reinterpret_cast<float4*>(tQK + swz_off4(t, 2 * q8 + 1, 128)) = x1;
-      bf16x8(stg + STG_K + t * 256 + q8 * 16, x0, x1);
-      *reinterpret_cast<float4*>(tQK + swz_off4(64 + t, 2 * q8, 128)) = x0;
-      *reinterpret_cast<float4*>(tQK + swz_off4(64 + t, 2 * q8 + 1, 128)) = x1;
-    }
     {
-      // k^T: thread c2 takes channel c2 of every token
-      const __nv_bfloat16* kst = reinterpret_cast<const __nv_bfloat16*>(stg + STG_K);
+      // q and k: 2048 groups of 8 bf16; all loads are issued before any store
+      uint4 raw[8];
 #pragma unroll
-      for (int jq = 0; jq < 16; ++jq) {
-        float4 x;
-        x.x = __bfloat162float(kst[(4 * jq + 0) * kDK + tid]);
-        x.y = __bfloat162float(kst[(4 * jq + 1) * kDK + tid]);
-        x.z = __bfloat162float(kst[(4 * jq + 2) * kDK + tid]);
-        x.w = __bfloat162float(kst[(4 * jq + 3) * kDK + tid]);
-        *reinterpret_cast<float4*>(tKT + swz_off4(tid, jq, 128)) = x;
+      for (int n = 0; n < 8; ++n) {
+        const int i = tid + kThreads * n;
+        const int t = (i >> 4) & 63, q8 = i & 15;
+        raw[n] = *reinterpret_cast<const uint4*>(stg + ((i >> 10) ? STG_K : STG_Q) + t * 256 + q8 * 16);
       }
-    }
+      const __nv_bfloat16* kst = reinterpret_cast<const __nv_bfloat16*>(stg + STG_K);
+      const int kc = tid & 127, jh = tid >> 7;
+      __nv_bfloat16 kcol[32];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int i = tid + kThreads * n;          // 256 groups of 8 bf16
-      const int j = i >> 2, q8 = i & 3;
+      for (int x = 0; x < 32; ++x) kcol[x] = kst[(jh * 32 + x) * kDK + kc];
+      const uint4 vraw = *reinterpret_cast<const uint4*>(stg + STG_V + (tid >> 2) * 64 + (tid & 3) * 16);
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const int i = tid + kThreads * n;
+        const int t = (i >> 4) & 63, q8 = i & 15, row = (i >> 10) * 64 + t;
+        float4 x0, x1;
+        bf16x8(reinterpret_cast<const unsigned char*>(&raw[n]), x0, x1);
+        *reinterpret_cast<float4*>(tQK + swz_off4(row, 2 * q8, 128)) = x0;
+        *reinterpret_cast<float4*>(tQK + swz_off4(row, 2 * q8 + 1, 128)) = x1;
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        *reinterpret_cast<float4*>(tKT + swz_off4(kc, jh * 8 + x, 128)) =
+            make_float4(__bfloat162float(kcol[4 * x]), __bfloat162float(kcol[4 * x + 1]),
+                        __bfloat162float(kcol[4 * x + 2]), __bfloat162float(kcol[4 * x + 3]));
       float4 x0, x1;
-      bf16x8(stg + STG_V + j * 64 + q8 * 16, x0, x1);
-      *reinterpret_cast<float4*>(tVF + swz_off4(j, 2 * q8, 64)) = x0;
-      *reinterpret_cast<float4*>(tVF + swz_off4(j, 2 * q8 + 1, 64)) = x1;
+      bf16x8(reinterpret_cast<const unsigned char*>(&vraw), x0, x1);
+      *reinterpret_cast<float4*>(tVF + swz_off4(tid >> 2, 2 * (tid & 3), 64)) = x0;
+      *reinterpret_cast<float4*>(tVF + swz_off4(tid >> 2, 2 * (tid & 3) + 1, 64)) = x1;
     }
     fence_smem_to_async();
     __syncthreads();
@@ -306,10 +320,10 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ---- 3. Gram [q; k] k^T on the tensor cores; meanwhile decay the state -----------------
     if (tid == 0) {
       fence_after_sync();
-      mma_chain(tb + TM_G, dQ, 128, dK, 128, kDK / 8, idesc_tf32(128, 64, false, false), false);
+      mma_chain(tb + TM_G, dQK, 128, dK, 128, kDK / 8, idesc_tf32(128, 64, false, false), false);
       mma_commit(mma_bar);
     }
-    {
+    if (tid < kDK) {
       float sd[kDVS];
       const float egc = ss.egc;
 #pragma unroll
@@ -320,127 +334,153 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if ((aborted = wait_bar(mma_bar, mphase))) break;
     // ---- 4. P (decayed, lower) and A (decayed, beta, strictly lower) --------------------------
     {
-      float d0[32], d1[32];
-      tmem_ld32(tb + tlane + TM_G, d0);
-      tmem_ld32(tb + tlane + TM_G + 32, d1);
+      // thread: Gram row r = 32 q4 + lane, columns 32 hw .. 32 hw + 31
+      float d[32], gj[32];
+      tmem_ld32(tb + tlane + TM_G + 32 * hw, d);
+#pragma unroll
+      for (int x = 0; x < 32; ++x) gj[x] = ss.g[32 * hw + x];
+      const int r = 32 * q4 + lane;
+      const int t = r & 63;
+      const float gt = ss.g[t];
+      const float bt = ss.beta[t];
       tmem_wait_ld();
-      const int r = tid & 63;
-      const float gt = ss.g[r];
-      if (tid < 64) {
+      if (r < 64) {
 #pragma unroll
-        for (int jq = 0; jq < 16; ++jq) {
-          float e[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int j = 4 * jq + x;
-            const float d = j < 32 ? d0[j] : d1[j - 32];
-            e[x] = j <= r ? d * __expf(gt - ss.g[j]) : 0.f;
-          }
-          st_tile4(tP, 64, r, jq, make_float4(e[0], e[1], e[2], e[3]));
+        for (int x = 0; x < 32; ++x) {
+          const int j = 32 * hw + x;
+          d[x] = j <= t ? d[x] * __expf(gt - gj[x]) : 0.f;
         }
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          st_tile4(tP, 64, t, 8 * hw + x, make_float4(d[4 * x], d[4 * x + 1], d[4 * x + 2], d[4 * x + 3]));
       } else {
-        const float bt = ss.beta[r];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float d = j < 32 ? d0[j] : d1[j - 32];
-          As[sx(r, j)] = j < r ? bt * d * __expf(gt - ss.g[j]) : 0.f;
+        for (int x = 0; x < 32; ++x) {
+          const int j = 32 * hw + x;
+          d[x] = j < t ? bt * d[x] * __expf(gt - gj[x]) : 0.f;
         }
+#pragma unroll
+        for (int x = 0; x < 32; ++x) As[sx(t, 32 * hw + x)] = d[x];
       }
     }
     __syncthreads();
     // ---- 5. X = (I + A)^{-1}: diagonal 16x16 blocks, then three block levels --------------------
-    if (tid < 64) {
-      const int a = tid >> 4, jl = tid & 15, base = 16 * a;
+    // Diagonal 16x16 blocks: warp a (a < 4) inverts block a, lane jl < 16 owning column
+    // jl.  In the sx() layout, entry (16a + tl, 16a + i) sits at
+    // (16a + tl) * 64 + (16a ^ (16a & 16)) + (i ^ tl): a compile-time offset from the
+    // block's base once tl and i are unrolled.
+    if (warp < 4 && lane < 16) {
+      const int base = 16 * warp, jl = lane;
+      const int bx = base ^ (base & 16);
+      const float* Ab = As + base * 64 + bx;
       float x[16];
 #pragma unroll
       for (int tl = 0; tl < 16; ++tl) {
-        float acc = (tl == jl) ? 1.f : 0.f;
+        float a_row[16];
 #pragma unroll
-        for (int i = 0; i < tl; ++i) acc = fmaf(-As[sx(base + tl, base + i)], x[i], acc);
-        x[tl] = (tl < jl) ? 0.f : acc;
+        for (int i = 0; i < tl; ++i) a_row[i] = Ab[tl * 64 + (i ^ tl)];
+        float acc0 = (tl == jl) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < tl; i += 2) {
+          acc0 = fmaf(-a_row[i], x[i], acc0);
+          if (i + 1 < tl) acc1 = fmaf(-a_row[i + 1], x[i + 1], acc1);
+        }
+        x[tl] = (tl < jl) ? 0.f : acc0 + acc1;
       }
+      float* Xb = Xs + base * 64 + bx;
 #pragma unroll
-      for (int tl = 0; tl < 16; ++tl) Xs[sx(base + tl, base + jl)] = x[tl];
+      for (int tl = 0; tl < 16; ++tl) Xb[tl * 64 + (jl ^ tl)] = x[tl];
     }
     __syncthreads();
+    // Off-diagonal blocks, level d = a - b: Z[b] = sum_{m=b}^{a-1} A[a][m] X[m][b], then
+    // X[a][b] = -X[a][a] Z[b].  Thread layout per 16x16 block: row r, columns 4cq..4cq+3;
+    // 64 threads per block, up to 3 blocks per level.
+    {
+      const int bb = tid >> 6, r = (tid >> 2) & 15, cq = tid & 3;
 #pragma unroll
-    for (int d = 1; d <= 3; ++d) {
-      const int nblk = 4 - d;
-      // Z[bb] = sum_{m=bb}^{bb+d-1} A[bb+d][m] X[m][bb]
+      for (int d = 1; d <= 3; ++d) {
+        const bool act = bb < 4 - d;
+        const int aa = bb + d;
+        if (act) {
+          float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
-      for (int n = 0; n < 2 * nblk; ++n) {
-        const int e = tid + kThreads * n;
-        const int bb = e >> 8, r = (e >> 4) & 15, cc = e & 15, aa = bb + d;
-        float z0 = 0.f, z1 = 0.f;
+          for (int m = 0; m < d; ++m) {
 #pragma unroll
-        for (int m = 0; m < d; ++m)
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const int mm = 16 * (bb + m);
-            z0 = fmaf(As[sx(16 * aa + r, mm + i)], Xs[sx(mm + i, 16 * bb + cc)], z0);
-            z1 = fmaf(As[sx(16 * aa + r, mm + i + 1)], Xs[sx(mm + i + 1, 16 * bb + cc)], z1);
+            for (int i = 0; i < 16; ++i) {
+              const int k = 16 * (bb + m) + i;
+              const float a = As[sx(16 * aa + r, k)];
+              float e[4];
+              ld4_sx(Xs, k, i & 3, 16 * bb + 4 * cq, e);
+              z0 = fmaf(a, e[0], z0);
+              z1 = fmaf(a, e[1], z1);
+              z2 = fmaf(a, e[2], z2);
+              z3 = fmaf(a, e[3], z3);
+            }
           }
-        Zs[bb * 256 + r * 16 + cc] = z0 + z1;
-      }
-      __syncthreads();
-      // X[bb+d][bb] = -X[bb+d][bb+d] Z[bb]
-#pragma unroll
-      for (int n = 0; n < 2 * nblk; ++n) {
-        const int e = tid + kThreads * n;
-        const int bb = e >> 8, r = (e >> 4) & 15, cc = e & 15, aa = bb + d;
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          x0 = fmaf(Xs[sx(16 * aa + r, 16 * aa + i)], Zs[bb * 256 + i * 16 + cc], x0);
-          x1 = fmaf(Xs[sx(16 * aa + r, 16 * aa + i + 1)], Zs[bb * 256 + (i + 1) * 16 + cc], x1);
+          *reinterpret_cast<float4*>(&Zs[bb * 256 + r * 16 + 4 * cq]) = make_float4(z0, z1, z2, z3);
         }
-        Xs[sx(16 * aa + r, 16 * bb + cc)] = -(x0 + x1);
+        __syncthreads();
+        if (act) {
+          float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float xa = Xs[sx(16 * aa + r, 16 * aa + i)];
+            const float4 zz = *reinterpret_cast<const float4*>(&Zs[bb * 256 + i * 16 + 4 * cq]);
+            x0 = fmaf(xa, zz.x, x0);
+            x1 = fmaf(xa, zz.y, x1);
+            x2 = fmaf(xa, zz.z, x2);
+            x3 = fmaf(xa, zz.w, x3);
+          }
+          const int row = 16 * aa + r, col = 16 * bb + 4 * cq;
+          Xs[sx(row, col + 0)] = -x0;
+          Xs[sx(row, col + 1)] = -x1;
+          Xs[sx(row, col + 2)] = -x2;
+          Xs[sx(row, col + 3)] = -x3;
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
     // ---- 6. T = X Diag(beta) as a tf32 operand (blocks above the diagonal are zero) -----------
     {
-      const int r = tid & 63, half = tid >> 6;
-      float xr[32];
+      const int r = tid & 63, qq = tid >> 6;      // 16 columns per thread
+      float xr[16];
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int j = half * 32 + x;
-        xr[x] = ((j >> 4) <= (r >> 4)) ? Xs[sx(r, j)] * ss.beta[j] : 0.f;
+      for (int x = 0; x < 16; ++x) {
+        const int j = qq * 16 + x;
+        xr[x] = (qq <= (r >> 4)) ? Xs[sx(r, j)] * ss.beta[j] : 0.f;
       }
       __syncthreads();   // X (which aliases T) fully read
 #pragma unroll
-      for (int x = 0; x < 8; ++x)
-        st_tile4(tTM, 64, r, half * 8 + x,
+      for (int x = 0; x < 4; ++x)
+        st_tile4(tTM, 64, r, qq * 4 + x,
                  make_float4(xr[4 * x], xr[4 * x + 1], xr[4 * x + 2], xr[4 * x + 3]));
     }
     fence_smem_to_async();
     fence_before_sync();
     __syncthreads();
-    // ---- 7. Y = K S0^T, O1 = Q S0^T ------------------------------------------------------------
+    // ---- 7. [O1; Y] = [Q; K] S0^T  (one M=128 product) ------------------------------------------
     if (tid == 0) {
       fence_after_sync();
-      const uint32_t i64x32 = idesc_tf32(64, 32, false, false);
-      mma_chain(tb + TM_Y, dK, 128, dSS, kDVS, kDK / 8, i64x32, false);
-      mma_chain(tb + TM_O1, dQ, 128, dSS, kDVS, kDK / 8, i64x32, false);
+      mma_chain(tb + TM_OY, dQK, 128, dSS, kDVS, kDK / 8, idesc_tf32(128, 32, false, false), false);
       mma_commit(mma_bar);
     }
     if ((aborted = wait_bar(mma_bar, mphase))) break;
-    // ---- 8. R = V - Diag(e^G) Y as the operand [v][j] ---------------------------------------------
-    {
+    // ---- 8. R = V - Diag(e^G) Y as the operand [v][j] (Y rows live in lanes 64-127) -------------
+    if (hw == 0 && q4 >= 2) {
+      const int j = 32 * (q4 - 2) + lane;
       float y[32];
-      tmem_ld32(tb + tlane + TM_Y, y);
-      tmem_wait_ld();
-      if (lane < 16) {
-        const int j = warp * 16 + lane;
-        const float eg = ss.eg[j];
+      float4 vx[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 vx = *reinterpret_cast<const float4*>(tVF + swz_off4(j, q, 64));
-          st_tile(tRT, kDVS, 4 * q + 0, j, fmaf(-eg, y[4 * q + 0], vx.x));
-          st_tile(tRT, kDVS, 4 * q + 1, j, fmaf(-eg, y[4 * q + 1], vx.y));
-          st_tile(tRT, kDVS, 4 * q + 2, j, fmaf(-eg, y[4 * q + 2], vx.z));
-          st_tile(tRT, kDVS, 4 * q + 3, j, fmaf(-eg, y[4 * q + 3], vx.w));
-        }
+      for (int q = 0; q < 8; ++q) vx[q] = *reinterpret_cast<const float4*>(tVF + swz_off4(j, q, 64));
+      const float eg = ss.eg[j];
+      tmem_ld32(tb + tlane + TM_OY, y);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        st_tile(tRT, kDVS, 4 * q + 0, j, fmaf(-eg, y[4 * q + 0], vx[q].x));
+        st_tile(tRT, kDVS, 4 * q + 1, j, fmaf(-eg, y[4 * q + 1], vx[q].y));
+        st_tile(tRT, kDVS, 4 * q + 2, j, fmaf(-eg, y[4 * q + 2], vx[q].z));
+        st_tile(tRT, kDVS, 4 * q + 3, j, fmaf(-eg, y[4 * q + 3], vx[q].w));
       }
     }
     fence_smem_to_async();
@@ -453,18 +493,18 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mma_commit(mma_bar);
     }
     if ((aborted = wait_bar(mma_bar, mphase))) break;
-    // ---- 10. U and U' = Diag(e^{G_last - G}) U as operands [v][j] ----------------------------------
+    // ---- 10. U and U' = Diag(e^{G_last - G}) U as operands [v][j] (M=64 rows: lanes 0-15) ---------
     {
-      float u[32];
-      tmem_ld32(tb + tlane + TM_U, u);
+      float u[16];
+      tmem_ld16(tb + tlane + TM_U + 16 * hw, u);
       tmem_wait_ld();
       if (lane < 16) {
-        const int j = warp * 16 + lane;
+        const int j = 16 * q4 + lane;
         const float el = ss.egl[j];
 #pragma unroll
-        for (int vv = 0; vv < kDVS; ++vv) {
-          st_tile(tUT, kDVS, vv, j, u[vv]);
-          st_tile(tUPT, kDVS, vv, j, u[vv] * el);
+        for (int x = 0; x < 16; ++x) {
+          st_tile(tUT, kDVS, 16 * hw + x, j, u[x]);
+          st_tile(tUPT, kDVS, 16 * hw + x, j, u[x] * el);
         }
       }
     }
@@ -479,47 +519,61 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mma_commit(mma_bar);
     }
     if ((aborted = wait_bar(mma_bar, mphase))) break;
-    // ---- 12. outputs and the new state ------------------------------------------------------------------
+    // ---- 12. new state (warps 0-3) and outputs O = Diag(e^G) O1 + O2 (warps 4-5) --------------------
     {
-      float o1[32], o2[32];
-      tmem_ld32(tb + tlane + TM_O1, o1);
-      tmem_ld32(tb + tlane + TM_O2, o2);
-      tmem_ld32(tb + tlane + TM_S, st);
+      float o2[16];
+      tmem_ld16(tb + tlane + TM_O2 + 16 * hw, o2);
       tmem_wait_ld();
       if (lane < 16) {
-        const int t = warp * 16 + lane;
-        if (t < L) {
-          const float eg = ss.eg[t];
-          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
-          if constexpr (sizeof(Tout) == 2) {
+        const int t = 16 * q4 + lane;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 pk;
-              __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
+        for (int x = 0; x < 16; ++x) Ox[t * 32 + ((16 * hw + x) ^ (t & 31))] = o2[x];
+      }
+      if (tid < kDK) {
+        tmem_ld32(tb + tlane + TM_S, st);
+        tmem_wait_ld();
 #pragma unroll
-              for (int x = 0; x < 4; ++x)
-                hp[x] = __floats2bfloat162_rn(fmaf(eg, o1[8 * q + 2 * x], o2[8 * q + 2 * x]),
-                                              fmaf(eg, o1[8 * q + 2 * x + 1], o2[8 * q + 2 * x + 1]));
-              reinterpret_cast<uint4*>(dst)[q] = pk;
-            }
-          } else {
+        for (int vv = 0; vv < kDVS; ++vv) st_tile(tSS, kDVS, vv, tid, st[vv]);
+      }
+    }
+    __syncthreads();
+    if (hw == 1 && q4 < 2) {
+      const int t = 32 * q4 + lane;
+      float o1[32];
+      tmem_ld32(tb + tlane + TM_OY, o1);
+      float o2[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<float4*>(dst)[q] =
-                  make_float4(fmaf(eg, o1[4 * q], o2[4 * q]), fmaf(eg, o1[4 * q + 1], o2[4 * q + 1]),
-                              fmaf(eg, o1[4 * q + 2], o2[4 * q + 2]),
-                              fmaf(eg, o1[4 * q + 3], o2[4 * q + 3]));
+      for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
+      tmem_wait_ld();
+      if (t < L) {
+        const float eg = ss.eg[t];
+        Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
+        if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 pk;
+            __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              hp[x] = __floats2bfloat162_rn(fmaf(eg, o1[8 * q + 2 * x], o2[8 * q + 2 * x]),
+                                            fmaf(eg, o1[8 * q + 2 * x + 1], o2[8 * q + 2 * x + 1]));
+            reinterpret_cast<uint4*>(dst)[q] = pk;
           }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(dst)[q] =
+                make_float4(fmaf(eg, o1[4 * q], o2[4 * q]), fmaf(eg, o1[4 * q + 1], o2[4 * q + 1]),
+                            fmaf(eg, o1[4 * q + 2], o2[4 * q + 2]),
+                            fmaf(eg, o1[4 * q + 3], o2[4 * q + 3]));
         }
       }
-#pragma unroll
-      for (int vv = 0; vv < kDVS; ++vv) st_tile(tSS, kDVS, vv, tid, st[vv]);
     }
     fence_smem_to_async();
     fence_before_sync();
     __syncthreads();
   }
-  if (!aborted && s_final) {
+  if (!aborted && s_final && tid < kDK) {
 #pragma unroll
     for (int vv = 0; vv < kDVS; ++vv) s_final[sbase + (long)(v0 + vv) * kDK + tid] = st[vv];
   }
