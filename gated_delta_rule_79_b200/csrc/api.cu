@@ -61,9 +61,9 @@ static gdr_status prefill(bool kda, const void* q, const void* k, const void* v,
     return fail(GDR_ERR_UNSUPPORTED, "%s: chunk=%d (only %d is supported)", fn, chunk, GDR_CHUNK);
   const size_t need = gdr_prefill_workspace_bytes(B, T, H, dk, dv, kda);
   if (need == 0) return fail(GDR_ERR_INVALID_ARG, "%s: sizes overflow", fn);
-  if (!workspace || ws_bytes < need)
-    return fail(GDR_ERR_INVALID_ARG, "%s: workspace %p of %zu bytes, need %zu", fn, workspace,
-                ws_bytes, need);
+  if (!workspace || ws_bytes < kStatusBytes)
+    return fail(GDR_ERR_INVALID_ARG, "%s: workspace %p of %zu bytes, need at least %zu", fn,
+                workspace, ws_bytes, kStatusBytes);
   if (((uintptr_t)workspace & 255u) != 0)
     return fail(GDR_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
   cudaStream_t st = (cudaStream_t)stream;

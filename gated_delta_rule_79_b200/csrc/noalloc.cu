@@ -53,7 +53,9 @@ extern "C" gdr_status gdn_prefill_noalloc(const void* q, const void* k, const vo
                                           void* o, float* s_final, int B, int T, int H, int dk,
                                           int dv, int in_dtype, int out_dtype, int chunk,
                                           void* stream) {
-  const size_t need = gdr_prefill_workspace_bytes(B, T, H, dk, dv, 0);
+  // The static scratch serves the single-kernel prefill, which needs the status word
+  // only; the faster two-kernel path would need gdr_prefill_workspace_bytes(...).
+  const size_t need = gdr_prefill_workspace_bytes(B, T, H, dk, dv, 0) ? kStatusBytes : 0;
   if (need > kNoAllocScratchBytes)
     return fail(GDR_ERR_INVALID_ARG,
                 "gdn_prefill_noalloc: these sizes need %zu bytes of scratch; the static "

@@ -616,9 +616,22 @@ bool tc_prefill_supported(const PrefillArgs& a) {
   return a.in_dtype == GDR_BF16 && a.dk == kDK && !a.kda && a.dv % kDVS == 0;
 }
 
-size_t tc_prefill_workspace(int, int, int, int, int, bool) { return 0; }
+size_t split_prefill_workspace(int B, int T, int H);            // prefill_split.cu
+cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
+
+// The two-kernel path (per-chunk prep over the whole GPU, then the carry) needs a
+// workspace of 33 KB per chunk; with a smaller workspace this single-kernel path runs.
+size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
+  PrefillArgs a{};
+  a.in_dtype = GDR_BF16;
+  a.dk = dk;
+  a.dv = dv;
+  a.kda = kda;
+  return tc_prefill_supported(a) ? split_prefill_workspace(B, T, H) : 0;
+}
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
+  if (a.ws_bytes >= 256 + split_prefill_workspace(a.B, a.T, a.H)) return launch_prefill_split(a, st);
   if (a.out_dtype == GDR_F32) return launch_t<float>(a, st);
   return launch_t<__nv_bfloat16>(a, st);
 }

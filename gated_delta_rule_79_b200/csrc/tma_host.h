@@ -25,9 +25,11 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map over a dense bf16 tensor [B, T, H, D] (D contiguous) whose boxes are
-// `box_d` x 1 head x `box_t` tokens x 1 batch; rows past T read as zero.
+// `box_d` x 1 head x `box_t` tokens x 1 batch; rows past T read as zero.  With
+// swizzle128 (box_d * 2 must then be 128 bytes) a box lands in shared memory as the
+// 128-byte swizzled K-major operand layout.
 inline bool encode_bthd_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int D,
-                             int box_d, int box_t) {
+                             int box_d, int box_t, bool swizzle128 = false) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -35,7 +37,8 @@ inline bool encode_bthd_bf16(CUtensorMap* m, const void* base, int B, int T, int
   cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -74,11 +74,14 @@ GDR_API int gdr_version(void);
  * into the library. */
 GDR_API const char* gdr_last_error(void);
 
-/* Bytes of device workspace that gdn_prefill / kda_prefill need for these
- * sizes (kda != 0 selects KDA).  The workspace holds the device status word of
- * the bounded waits and the per-chunk exchange area of the prefill kernels.  It
- * must be zero-filled once when allocated; the library leaves it ready for the
- * next call.  Returns 0 when the sizes are invalid. */
+/* Bytes of device workspace with which gdn_prefill / kda_prefill run their
+ * fastest path for these sizes (kda != 0 selects KDA); 0 when the sizes are
+ * invalid.  The workspace holds the device status word of the bounded waits
+ * (the first 256 bytes) and, for the bf16 GDN two-kernel prefill, 33 KB per
+ * chunk of 64 tokens per (sequence, head) of precomputed chunk operands.  Any
+ * workspace of at least 256 bytes is accepted: with less than the returned size
+ * the single-kernel path runs.  It must be zero-filled once when allocated; the
+ * library leaves it ready for the next call. */
 GDR_API size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, int kda);
 
 /* Chunked prefill: runs the recurrence over T tokens for B sequences and H heads
@@ -94,8 +97,8 @@ GDR_API size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, 
  *   s_final  [B, H, d_v, d_k] fp32 (written), or NULL to skip; may be the same
  *            pointer as s0 (in-place carry), must not otherwise overlap inputs
  *   chunk    must be GDR_CHUNK (64)
- *   workspace, ws_bytes: at least gdr_prefill_workspace_bytes(...) bytes,
- *            zero-filled at allocation, 256-byte aligned
+ *   workspace, ws_bytes: at least 256 bytes (gdr_prefill_workspace_bytes(...)
+ *            for the fastest path), zero-filled at allocation, 256-byte aligned
  * B, T or H equal to 0 is a valid empty call (with T == 0, s_final receives s0,
  * or zeros when s0 is NULL).  in_dtype GDR_F32 runs the fp32 CUDA-core kernel;
  * GDR_BF16 runs the tensor-core kernel where one exists for (d_k, d_v). */
@@ -141,8 +144,9 @@ GDR_API gdr_status kda_decode(const void* q, const void* k, const void* v,
  * and embedders whose device memory is owned by another allocator under a fixed
  * budget.  Arguments, results and errors are those of gdn_prefill without the
  * workspace: the library uses a static device array of 4096 bytes instead,
- * reserved on every GPU that loads the library until the process exits.  Sizes
- * that would need more scratch are rejected with GDR_ERR_INVALID_ARG.  The
+ * reserved on every GPU that loads the library until the process exits, which
+ * runs the single-kernel prefill (it needs the 256-byte status word only).
+ * Sizes that would need more scratch are rejected with GDR_ERR_INVALID_ARG.  The
  * first call on a device looks up the array's device address with the device
  * current, so make that first call before any stream capture.  The call
  * allocates nothing and clears the array's status word after launching, so

@@ -14,12 +14,14 @@ from synth import Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_reports_timeout_and_recovers():
+@pytest.mark.parametrize("path", ["single-kernel", "two-kernel"])
+def test_bounded_wait_reports_timeout_and_recovers(path):
     import gated_delta_rule_79_b200 as g
     w = Workload("fi", "gdn", 1, 2, 100, 128, 128, "bf16", "randn")
     x = {k: v.cuda() for k, v in make_inputs(w, seed=11).items()}
     assert g.prefill_path(128, 128, torch.bfloat16, False) == "tensor-core"
-    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    full = g.lib.gdr_prefill_workspace_bytes(1, 100, 2, 128, 128, 0)
+    ws = torch.zeros(4096 if path == "single-kernel" else full, dtype=torch.uint8, device="cuda")
     old = os.environ.get("GDR_SPIN_LIMIT")
     os.environ["GDR_SPIN_LIMIT"] = "0"
     try:
