@@ -83,12 +83,13 @@ __device__ __forceinline__ void st_tile4(unsigned char* tile, int rows, int r, i
 
 constexpr int P_THREADS = 128;
 constexpr int P_QK = 0;                    // bf16 [128][128] SW128 (q rows 0-63, k 64-127)  32 KB
+// once the Gram has been read, the solve's scratch reuses the q/k tile:
+constexpr int P_X = 0;                     //   X scratch, sx() layout                        16 KB
+constexpr int P_A = 16384;                 //   packed strictly-lower A                       10 KB
+constexpr int P_Z = P_A + 10240;           //   level scratch [3][16][16]                      3 KB
 constexpr int P_OUT = 32768;               // P | T | gates: the chunk's workspace image      33 KB
-constexpr int P_X = P_OUT + 34816;         // X scratch, sx() layout                          16 KB
-constexpr int P_A = P_X + 16384;           // packed strictly-lower A                         10 KB
-constexpr int P_Z = P_A + 10240;           // level scratch [3][16][16]                        3 KB
-constexpr int P_SMALL = P_Z + 3072;
-constexpr int P_SMEM = P_SMALL + 1024 + 1024;
+constexpr int P_SMALL = P_OUT + 34816;
+constexpr int P_SMEM = P_SMALL + 1024 + 1024;   // 68 KB: three CTAs per SM
 constexpr uint32_t P_TM_COLS = 64;
 
 struct PrepSmall {
@@ -370,21 +371,28 @@ constexpr int C_RT = C_SSL + 8192;              // fp32 [32 v][64 j]; P U exchan
 constexpr int C_UT = C_RT + 8192;               // fp32 [32 v][64 j]                      8 KB
 constexpr int C_UPH = C_UT + 8192;              // bf16 [32 v][64 j] (e^{G_last-G} U) hi  4 KB
 constexpr int C_UPL = C_UPH + 4096;             //                                  lo    4 KB
-constexpr int C_SMALL = C_UPL + 4096;
-constexpr int C_SMEM = C_SMALL + 256 + 1024;
+constexpr int C_OX = C_UPL + 4096;              // P U exchange [64 t][32 v] (loader)    8 KB
+constexpr int C_SMALL = C_OX + 8192;
+constexpr int C_SMEM = C_SMALL + 1024 + 1024;
 static_assert(C_SMEM <= 232448, "shared memory");
 
-constexpr uint32_t TM_OY = 0;    // [q; k] S0^T, M=128 x 32: rows 0-63 O1, 64-127 Y
-constexpr uint32_t TM_U = 32;    // U, M=64 x 32
-constexpr uint32_t TM_O2 = 64;   // P U, M=64 x 32
-constexpr uint32_t TM_S = 96;    // S^T, M=128 x 32
-constexpr uint32_t C_TM_COLS = 128;
+// [q; k] S0^T (M=128 x 32: rows 0-63 O1, rows 64-127 Y) and P U (M=64 x 32) are
+// double-buffered by chunk parity: the loader warpgroup reads chunk c's outputs while
+// the carry already runs chunk c+1.
+constexpr uint32_t TM_OY = 0;    // + 32 * (c & 1)
+constexpr uint32_t TM_O2 = 64;   // + 32 * (c & 1)
+constexpr uint32_t TM_U = 128;   // U, M=64 x 32
+constexpr uint32_t TM_S = 160;   // S^T, M=128 x 32
+constexpr uint32_t C_TM_COLS = 256;
 
 struct CarrySmall {
   unsigned long long full[C_STAGES];    // TMA + bulk copy landed
   unsigned long long ready[C_STAGES];   // k^T built, stage ready for the carry
   unsigned long long empty[C_STAGES];   // carry done with the stage
   unsigned long long mma_bar;
+  unsigned long long out_full[2];   // chunk's O1 and P U are in TMEM (carry -> loader)
+  unsigned long long out_empty[2];  // loader has read them (loader -> carry)
+  float eg_out[2][64];              // e^{G_t} of the chunk whose outputs are pending
   uint32_t tmem;
   int abort;
 };
@@ -412,7 +420,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
   unsigned char* tUT = sm + C_UT;
   unsigned char* tUPH = sm + C_UPH;
   unsigned char* tUPL = sm + C_UPL;
-  float* Ox = reinterpret_cast<float*>(tRT);   // P U exchange [64 t][32 v], row-XOR layout
+  float* Ox = reinterpret_cast<float*>(sm + C_OX);   // P U exchange [64 t][32 v], row-XOR
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3;
@@ -429,6 +437,10 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(reinterpret_cast<uint64_t*>(&cs.empty[s]), 1);
     }
     mbar_init(reinterpret_cast<uint64_t*>(&cs.mma_bar), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_full[s]), 1);
+      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_empty[s]), 1);
+    }
     cs.abort = 0;
     fence_mbar_init();
   }
@@ -453,6 +465,65 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp >= 4) {
     // =========================== loader warpgroup =====================================
     const int lt = tid - 128;
+    // O = Diag(e^G) O1 + P U for chunk cc, read from the chunk's TMEM buffers once the
+    // carry has finished it; returns false on abort.
+    auto write_outputs = [&](int cc) -> bool {
+      const int ob = cc & 1;
+      const uint32_t use = (uint32_t)(cc >> 1);
+      uint64_t* ofull = reinterpret_cast<uint64_t*>(&cs.out_full[ob]);
+      if (lt == 0 && !mbar_wait(ofull, use & 1u, spin_limit)) give_up(ofull, use & 1u, false);
+      named_bar(2, 128);
+      if (cs.abort) return false;
+      fence_after_sync();
+      const int t0 = cc * kC;
+      const int L = min(kC, T - t0);
+      {
+        float o2[32];
+        tmem_ld32(tb + tlane + TM_O2 + 32 * ob, o2);
+        tmem_wait_ld();
+        if (lane < 16) {
+          const int t = 16 * q4 + lane;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) Ox[t * 32 + (x ^ (t & 31))] = o2[x];
+        }
+      }
+      named_bar(2, 128);
+      if (q4 < 2) {
+        const int t = 32 * q4 + lane;
+        float o1[32], o2[32];
+        tmem_ld32(tb + tlane + TM_OY + 32 * ob, o1);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
+        const float eg = cs.eg_out[ob][t];
+        tmem_wait_ld();
+        if (t < L) {
+          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
+          if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 pk;
+              __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                hp[x] = __floats2bfloat162_rn(fmaf(eg, o1[8 * q + 2 * x], o2[8 * q + 2 * x]),
+                                              fmaf(eg, o1[8 * q + 2 * x + 1], o2[8 * q + 2 * x + 1]));
+              reinterpret_cast<uint4*>(dst)[q] = pk;
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              reinterpret_cast<float4*>(dst)[q] =
+                  make_float4(fmaf(eg, o1[4 * q], o2[4 * q]), fmaf(eg, o1[4 * q + 1], o2[4 * q + 1]),
+                              fmaf(eg, o1[4 * q + 2], o2[4 * q + 2]),
+                              fmaf(eg, o1[4 * q + 3], o2[4 * q + 3]));
+          }
+        }
+      }
+      fence_before_sync();
+      named_bar(2, 128);
+      if (lt == 0) mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_empty[ob]));
+      return true;
+    };
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const uint32_t use = (uint32_t)(c >> 1);
@@ -504,7 +575,9 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       fence_smem_to_async();
       named_bar(2, 128);
       if (lt == 0) mbar_arrive(ready);
+      if (c > 0 && !write_outputs(c - 1)) break;
     }
+    if (!cs.abort) write_outputs(nchunks - 1);
   } else {
     // =========================== carry warpgroup ======================================
     // state: thread c < 128 owns row c of S^T (S[v0 + v][c], v < 32)
@@ -554,6 +627,12 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       if ((aborted = cs.abort != 0)) break;
       fence_after_sync();
       // ---- decay the state in TMEM, then [O1; Y] = [Q; K] (S_hi + S_lo)^T ----------------
+      const int ob = c & 1;
+      if (c >= 2 && tid == 0) {
+        uint64_t* oe = reinterpret_cast<uint64_t*>(&cs.out_empty[ob]);
+        const uint32_t par = (uint32_t)((c >> 1) - 1) & 1u;
+        if (!mbar_wait(oe, par, spin_limit)) give_up(oe, par, false);
+      }
       {
         float sd[kDVS];
         const float egc = gates[128];
@@ -564,16 +643,18 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       fence_before_sync();
       named_bar(1, 128);
+      // after the barrier: thread 0 has seen the loader free this output buffer
+      if (tid < 64) cs.eg_out[ob][tid] = gates[tid];
       if (tid == 0) {
         fence_after_sync();
         const uint64_t dQK = sdesc(a + S_QK, 16, 1024);
         const uint32_t id = idesc_bf16(128, 32);
 #pragma unroll
         for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16(tb + TM_OY, kstep(dQK, 128, ks), kstep(dSSH, kDVS, ks), id, ks > 0);
+          mma_bf16(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSH, kDVS, ks), id, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16(tb + TM_OY, kstep(dQK, 128, ks), kstep(dSSL, kDVS, ks), id, true);
+          mma_bf16(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSL, kDVS, ks), id, true);
         mma_commit(mma_bar);
       }
       if ((aborted = wait_mma())) break;
@@ -594,7 +675,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
         const float eg = gates[j];
-        tmem_ld32(tb + tlane + TM_OY, y);
+        tmem_ld32(tb + tlane + TM_OY + 32 * ob, y);
         tmem_wait_ld();
 #pragma unroll
         for (int v = 0; v < kDVS; ++v)
@@ -644,7 +725,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t it = idesc_tf32(64, 32, false, false);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_O2, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), it, ks > 0);
+          mma_tf32(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), it, ks > 0);
         const uint32_t ib = idesc_bf16(128, 32);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
@@ -654,54 +735,15 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_bf16(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPL, kDVS, ks), ib, true);
         mma_commit(mma_bar);
       }
-      const float eg_t = (tid < 64) ? gates[tid] : 0.f;   // read before the stage is released
       if ((aborted = wait_mma())) break;
-      if (tid == 0) mbar_arrive(reinterpret_cast<uint64_t*>(&cs.empty[s]));
-      // ---- new state; P U through shared memory; O = Diag(e^G) O1 + P U -------------------------
-      {
-        float o2[32];
-        tmem_ld32(tb + tlane + TM_O2, o2);
-        tmem_ld32(tb + tlane + TM_S, st);
-        tmem_wait_ld();
-        if (lane < 16) {
-          const int t = 16 * q4 + lane;
-#pragma unroll
-          for (int x = 0; x < 32; ++x) Ox[t * 32 + (x ^ (t & 31))] = o2[x];
-        }
-        write_state_operand();
+      if (tid == 0) {
+        mbar_arrive(reinterpret_cast<uint64_t*>(&cs.empty[s]));
+        mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
       }
-      fence_before_sync();
-      named_bar(1, 128);
-      if (q4 < 2) {
-        const int t = 32 * q4 + lane;
-        float o1[32], o2[32];
-        tmem_ld32(tb + tlane + TM_OY, o1);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
-        tmem_wait_ld();
-        if (t < L) {
-          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
-          if constexpr (sizeof(Tout) == 2) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 pk;
-              __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                hp[x] = __floats2bfloat162_rn(fmaf(eg_t, o1[8 * q + 2 * x], o2[8 * q + 2 * x]),
-                                              fmaf(eg_t, o1[8 * q + 2 * x + 1], o2[8 * q + 2 * x + 1]));
-              reinterpret_cast<uint4*>(dst)[q] = pk;
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<float4*>(dst)[q] =
-                  make_float4(fmaf(eg_t, o1[4 * q], o2[4 * q]), fmaf(eg_t, o1[4 * q + 1], o2[4 * q + 1]),
-                              fmaf(eg_t, o1[4 * q + 2], o2[4 * q + 2]),
-                              fmaf(eg_t, o1[4 * q + 3], o2[4 * q + 3]));
-          }
-        }
-      }
+      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
+      tmem_ld32(tb + tlane + TM_S, st);
+      tmem_wait_ld();
+      write_state_operand();
       fence_smem_to_async();
       fence_before_sync();
       named_bar(1, 128);
