@@ -555,6 +555,8 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!mbar_wait(full, use & 1u, spin_limit)) give_up(full, use & 1u, true);
       named_bar(2, 128);
       if (cs.abort) break;
+      // the loader forms this chunk's outputs later: keep its e^{G_t}
+      if (lt < 64) cs.eg_out[s][lt] = reinterpret_cast<const float*>(st + S_PT + WS_G)[lt];
       // k^T: thread lt takes channel lt of every token of the chunk
       {
         const unsigned char* qk = st + S_QK;
@@ -643,8 +645,6 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       fence_before_sync();
       named_bar(1, 128);
-      // after the barrier: thread 0 has seen the loader free this output buffer
-      if (tid < 64) cs.eg_out[ob][tid] = gates[tid];
       if (tid == 0) {
         fence_after_sync();
         const uint64_t dQK = sdesc(a + S_QK, 16, 1024);
@@ -739,8 +739,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (tid == 0) {
         mbar_arrive(reinterpret_cast<uint64_t*>(&cs.empty[s]));
         mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
-      }
-      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
+      }      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
       tmem_ld32(tb + tlane + TM_S, st);
       tmem_wait_ld();
       write_state_operand();
