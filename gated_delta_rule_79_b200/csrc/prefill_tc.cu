@@ -612,12 +612,15 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+// Both mixers take the tensor-core path for bf16 inputs with d_k = 128 and d_v a
+// multiple of 32; the rest runs on the CUDA cores.
 bool tc_prefill_supported(const PrefillArgs& a) {
-  return a.in_dtype == GDR_BF16 && a.dk == kDK && !a.kda && a.dv % kDVS == 0;
+  return a.in_dtype == GDR_BF16 && a.dk == kDK && a.dv % kDVS == 0;
 }
 
 size_t split_prefill_workspace(int B, int T, int H);            // prefill_split.cu
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_kda_tc(const PrefillArgs& a, cudaStream_t stream);  // prefill_kda_tc.cu
 
 // The two-kernel path (per-chunk prep over the whole GPU, then the carry) needs a
 // workspace of 33 KB per chunk; with a smaller workspace this single-kernel path runs.
@@ -627,10 +630,11 @@ size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
   a.dk = dk;
   a.dv = dv;
   a.kda = kda;
-  return tc_prefill_supported(a) ? split_prefill_workspace(B, T, H) : 0;
+  return tc_prefill_supported(a) && !kda ? split_prefill_workspace(B, T, H) : 0;
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
+  if (a.kda) return launch_prefill_kda_tc(a, st);
   if (a.ws_bytes >= 256 + split_prefill_workspace(a.B, a.T, a.H)) return launch_prefill_split(a, st);
   if (a.out_dtype == GDR_F32) return launch_t<float>(a, st);
   return launch_t<__nv_bfloat16>(a, st);
