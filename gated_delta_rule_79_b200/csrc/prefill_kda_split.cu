@@ -1,0 +1,788 @@
+// Kimi Delta Attention chunked prefill in two kernels (sm_100a, tcgen05 + TMA).
+//
+// "Super Apriel: One Checkpoint, Many Speeds", §2A names the KDA mixer: the delta
+// rule with one gate per key channel.  For a chunk of C = 64 tokens entering with
+// state S0 and the chunk-local cumulative log gate G[t][c] = sum_{s<=t} log alpha_s[c]:
+//
+//   A[t,j] = beta_t sum_c k_tc k_jc e^{G_tc - G_jc}  (j < t)
+//   P[t,j] =        sum_c q_tc k_jc e^{G_tc - G_jc}  (j <= t)
+//   T = (I + A)^{-1} Diag(beta)
+//   [O1; Y] = [Q (.) e^G; K (.) e^G] S0^T,  R = V - Y,  U = T R
+//   O = O1 + P U
+//   S^T <- Diag(e^{G_last}) S0^T + (K (.) e^{G_last - G})^T U
+//
+// Everything except the last three lines is independent of the state.
+// kda_chunk_prep_kernel computes it for every chunk of every head at once, two
+// CTAs per SM, and leaves per chunk, in the workspace, the operand tiles of the
+// carry as tf32 images in the tensor cores' shared-memory layout:
+//   group A: [Q (.) e^G; K (.) e^G] (128 x 128) and e^{G_last} (128 floats)
+//   group C: T (64 x 64)
+//   group D: (K (.) e^{G_last - G})^T (128 x 64) and P (64 x 64)
+// kda_chunk_carry_kernel then walks the chunks of each (head, 32-wide value slice).
+// Its loader warpgroup only copies: each group has its own full/empty barrier pair
+// and is refilled for the next chunk as soon as the product that reads it has
+// completed, so one buffer per group keeps the carry fed.  The loader also forms
+// the outputs O = O1 + P U of the previous chunk.
+//
+// The decayed Gram factors through a per-channel reference Gm_c halfway between
+// the chunk's first and last G:  e^{G_tc - G_jc} = e^{G_tc - Gm_c} e^{Gm_c - G_jc},
+// one tf32 product of L = [Q; K] (.) e^{G - Gm} and R = K (.) e^{Gm - G}.  Both
+// factors stay normal fp32 numbers while the channel's log gate drops by at most
+// kMaxSpan over the chunk; wider channels are left out of the product and their
+// terms are added exactly on the CUDA cores.
+//
+// Precision: all products run as kind::tf32 with operands rounded to nearest.  Waits
+// are bounded; a give-up records GDR_ERR_TIMEOUT in the workspace status word,
+// drains what was issued, frees tensor memory and ends the CTA.
+
+#include <math.h>
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+#include "tma_host.h"
+
+namespace gdr {
+namespace {
+
+using namespace tc;
+
+constexpr int kC = GDR_CHUNK;
+constexpr int kDK = 128;
+constexpr int kDVS = 32;
+constexpr float kMaxSpan = 168.f;
+constexpr uint32_t kDrainLimit = 1u << 26;
+constexpr size_t kStatusBytes = 256;
+
+// Workspace image of one chunk (bytes).
+constexpr int WS_QK = 0;                   // [Q~; K~] tf32 SW128, 128 rows x 128     64 KB
+constexpr int WS_EGL = 65536;              // e^{G_last} per channel                 512 B
+constexpr int WS_A_BYTES = 66048;
+constexpr int WS_T = WS_A_BYTES;           // T tf32 SW128, 64 x 64                   16 KB
+constexpr int WS_KH = WS_T + 16384;        // K^ tf32 SW128, 128 rows (c) x 64 (j)    32 KB
+constexpr int WS_P = WS_KH + 32768;        // P tf32 SW128, 64 x 64                   16 KB
+constexpr int WS_D_BYTES = 32768 + 16384;
+constexpr int kChunkWs = WS_P + 16384;     // 131584
+
+__device__ __forceinline__ int sx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+
+__device__ __forceinline__ void ld4_sx(const float* base, int k, int klo, int c4, float (&e)[4]) {
+  const float4 f = *reinterpret_cast<const float4*>(base + k * 64 + (c4 ^ (k & 28)));
+  const float v[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+  for (int x = 0; x < 4; ++x) e[x] = v[x ^ klo];
+}
+
+__device__ __forceinline__ uint64_t kstep(uint64_t desc0, int rows, int ks) {
+  return desc0 + (uint64_t)((((ks >> 2) * rows * 128) + ((ks & 3) * 32)) >> 4);
+}
+
+__device__ __forceinline__ void st_tile(unsigned char* tile, int rows, int r, int c, float x) {
+  *reinterpret_cast<float*>(tile + swz_off(r, c, rows)) = to_tf32(x);
+}
+
+__device__ __forceinline__ float4 tf32x4(float a, float b, float c, float d) {
+  return make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
+
+// ========================================================================================
+// Kernel 1: per-chunk operand images
+// ========================================================================================
+
+constexpr int P_THREADS = 256;
+constexpr int P_L = 0;            // L = [Q; K] (.) e^{G - Gm}, tf32 [128][128] SW128      64 KB
+                                  //   after the Gram: A (sx) | X (sx) | level scratch
+constexpr int P_AS = 0, P_XS = 16384, P_ZS = 32768;
+constexpr int P_R = 65536;        // R = K (.) e^{Gm - G}, tf32 [64][128] SW128            32 KB
+                                  //   after the Gram: G [64 t][128 c] for wide channels
+constexpr int P_SMALL = P_R + 32768;
+constexpr int P_SMEM = P_SMALL + 3072 + 1024;   // about 100 KB: two CTAs per SM
+constexpr uint32_t P_TM_G = 0;    // Gram, M=128 x 64
+constexpr uint32_t P_TM_GS = 64;  // G by channel: lane c, columns t
+constexpr uint32_t P_TM_COLS = 128;
+
+struct PrepSmall {
+  float beta[kC];
+  double tot[2][kDK];   // per channel: sum of the log gates of tokens 0-31 and 32-63
+  float g0[kDK];        // per channel: G of token 0
+  unsigned wmask[4];    // wide channels
+  uint32_t tmem;
+  unsigned long long mma_bar;
+};
+static_assert(sizeof(PrepSmall) <= 3072, "prep small");
+
+__global__ void __launch_bounds__(P_THREADS, 2)
+kda_chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                      const float* __restrict__ alpha, const float* __restrict__ beta,
+                      unsigned char* __restrict__ ws, int T, int H, int nchunks,
+                      unsigned int* __restrict__ status, uint32_t spin_limit) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sm = smem_raw + padb;
+  unsigned char* tL = sm + P_L;
+  unsigned char* tR = sm + P_R;
+  float* As = reinterpret_cast<float*>(sm + P_AS);
+  float* Xs = reinterpret_cast<float*>(sm + P_XS);
+  float* Zs = reinterpret_cast<float*>(sm + P_ZS);
+  float* Gw = reinterpret_cast<float*>(tR);
+  PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, hw = warp >> 2;
+  const int c = blockIdx.x % nchunks;
+  const int bh = blockIdx.x / nchunks;
+  const int h = bh % H, b = bh / H;
+  const int t0 = c * kC;
+  const int L = min(kC, T - t0);
+  const long row0 = ((long)b * T + t0) * H + h;    // token t of the chunk: row0 + t * H
+  unsigned char* img = ws + kStatusBytes + ((size_t)bh * nchunks + c) * kChunkWs;
+
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&ps.tmem, P_TM_COLS);
+  // ---- 1. this thread's channel cc, tokens 32 hw .. 32 hw + 31 (rows past T: alpha 1, 0)
+  const int cc = 32 * q4 + lane;
+  float g[32];
+  uint32_t qp[16], kp[16];   // bf16 pairs: tokens (2i, 2i+1) of the half
+  {
+    const unsigned short* qs = reinterpret_cast<const unsigned short*>(q);
+    const unsigned short* ks = reinterpret_cast<const unsigned short*>(k);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint32_t qa = 0, qb = 0, ka = 0, kb = 0;
+      const int ta = 32 * hw + 2 * i, tb2 = ta + 1;
+      if (ta < L) {
+        const long e = (row0 + (long)ta * H) * kDK + cc;
+        g[2 * i] = __ldg(alpha + e);
+        qa = __ldg(qs + e);
+        ka = __ldg(ks + e);
+      } else {
+        g[2 * i] = 1.f;
+      }
+      if (tb2 < L) {
+        const long e = (row0 + (long)tb2 * H) * kDK + cc;
+        g[2 * i + 1] = __ldg(alpha + e);
+        qb = __ldg(qs + e);
+        kb = __ldg(ks + e);
+      } else {
+        g[2 * i + 1] = 1.f;
+      }
+      qp[i] = qa | (qb << 16);
+      kp[i] = ka | (kb << 16);
+    }
+  }
+  if (tid < kC) ps.beta[tid] = tid < L ? beta[row0 + (long)tid * H] : 0.f;
+  // ---- 2. cumulative log gate: fp64 prefix over each half, halves joined by their sums
+  {
+    double acc = 0.0;
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      acc += (double)log_gate_accurate(g[x]);
+      g[x] = (float)acc;
+    }
+    ps.tot[hw][cc] = acc;
+    if (hw == 0) ps.g0[cc] = g[0];
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = ps.tmem;
+  const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
+  const double tot0 = ps.tot[0][cc];
+  if (hw == 1) {
+#pragma unroll
+    for (int x = 0; x < 32; ++x) g[x] = (float)(tot0 + (double)g[x]);
+  }
+  const float glast = (float)(tot0 + ps.tot[1][cc]);
+  const float g0c = ps.g0[cc];
+  const float gm = 0.5f * (g0c + glast);
+  const bool wc = (g0c - glast) > kMaxSpan;
+  if (hw == 0) {
+    const unsigned wm = __ballot_sync(0xffffffffu, wc);
+    if (lane == 0) ps.wmask[q4] = wm;
+  }
+  tmem_st32(tb + tlane + P_TM_GS + 32 * hw, g);
+  // ---- 3. Gram factors ----------------------------------------------------------------
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int x = 2 * i + u, t = 32 * hw + x;
+      const float qv = u ? bf16_hi(qp[i]) : bf16_lo(qp[i]);
+      const float kv = u ? bf16_hi(kp[i]) : bf16_lo(kp[i]);
+      const float e = wc ? 0.f : __expf(g[x] - gm);
+      const float ei = wc ? 0.f : __expf(gm - g[x]);
+      st_tile(tL, 128, t, cc, qv * e);
+      st_tile(tL, 128, 64 + t, cc, kv * e);
+      st_tile(tR, 64, t, cc, kv * ei);
+    }
+  }
+  tmem_wait_st();
+  fence_smem_to_async();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const bool anywide = (ps.wmask[0] | ps.wmask[1] | ps.wmask[2] | ps.wmask[3]) != 0u;
+  if (tid == 0) {
+    const uint64_t dL = sdesc(smem_u32(tL), 16, 1024), dR = sdesc(smem_u32(tR), 16, 1024);
+    const uint32_t id = idesc_tf32(128, 64, false, false);
+#pragma unroll 4
+    for (int ks = 0; ks < kDK / 8; ++ks)
+      mma_tf32(tb + P_TM_G, kstep(dL, 128, ks), kstep(dR, 64, ks), id, ks > 0);
+    mma_commit(mma_bar);
+  }
+  // ---- 4. while the Gram runs: the carry's [Q~; K~], e^{G_last} and K^ images -------------
+  {
+    unsigned char* iqk = img + WS_QK;
+    float kh[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int x = 2 * i + u, t = 32 * hw + x;
+        const float qv = u ? bf16_hi(qp[i]) : bf16_lo(qp[i]);
+        const float kv = u ? bf16_hi(kp[i]) : bf16_lo(kp[i]);
+        const float e = __expf(g[x]);
+        *reinterpret_cast<float*>(iqk + swz_off(t, cc, 128)) = to_tf32(qv * e);
+        *reinterpret_cast<float*>(iqk + swz_off(64 + t, cc, 128)) = to_tf32(kv * e);
+        kh[x] = t < L ? kv * __expf(fminf(glast - g[x], 0.f)) : 0.f;
+      }
+    }
+    if (hw == 0) reinterpret_cast<float*>(img + WS_EGL)[cc] = __expf(glast);
+    unsigned char* ikh = img + WS_KH;
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+      *reinterpret_cast<float4*>(ikh + swz_off4(cc, 8 * hw + x, 128)) =
+          tf32x4(kh[4 * x], kh[4 * x + 1], kh[4 * x + 2], kh[4 * x + 3]);
+  }
+  bool failed = false;
+  if (!mbar_wait(mma_bar, 0, spin_limit)) {
+    mbar_wait(mma_bar, 0, kDrainLimit);
+    failed = true;
+  }
+  fence_after_sync();
+  if (__syncthreads_or(failed)) {
+    if (lane == 0) atomicOr(status, 1u);
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
+    return;
+  }
+  if (anywide) {
+    // G as [64 t][128 c] in the (now free) R area, for the exact terms
+    float gg[32];
+    tmem_ld32(tb + tlane + P_TM_GS + 32 * hw, gg);
+    tmem_wait_ld();
+#pragma unroll
+    for (int x = 0; x < 32; ++x) Gw[(32 * hw + x) * kDK + cc] = gg[x];
+    __syncthreads();
+  }
+  // ---- 5. P (lower) to the image; A (beta, strictly lower) to the solve's scratch -----------
+  {
+    float d[32];
+    tmem_ld32(tb + tlane + P_TM_G + 32 * hw, d);
+    const int r = 32 * q4 + lane;      // Gram row: q rows 0-63, k rows 64-127
+    const int t = r & 63;
+    const float bt = ps.beta[t];
+    tmem_wait_ld();
+    if (anywide) {
+      const __nv_bfloat16* xs = r < 64 ? q : k;
+#pragma unroll 1
+      for (int w = 0; w < 4; ++w) {
+        unsigned m = ps.wmask[w];
+        while (m) {
+          const int ch = 32 * w + __ffs(m) - 1;
+          m &= m - 1;
+          const float xv = t < L ? __bfloat162float(xs[(row0 + (long)t * H) * kDK + ch]) : 0.f;
+          const float gt = Gw[t * kDK + ch];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int j = 32 * hw + x;
+            if (j <= t && j < L)
+              d[x] += xv * __bfloat162float(k[(row0 + (long)j * H) * kDK + ch]) *
+                      __expf(gt - Gw[j * kDK + ch]);
+          }
+        }
+      }
+    }
+    if (r < 64) {
+      unsigned char* ip = img + WS_P;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        float e[4];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) e[y] = (32 * hw + 4 * x + y) <= t ? d[4 * x + y] : 0.f;
+        *reinterpret_cast<float4*>(ip + swz_off4(t, 8 * hw + x, 64)) = tf32x4(e[0], e[1], e[2], e[3]);
+      }
+    } else {
+#pragma unroll
+      for (int x = 0; x < 32; ++x) As[sx(t, 32 * hw + x)] = (32 * hw + x) < t ? bt * d[x] : 0.f;
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
+  // ---- 6. X = (I + A)^{-1}: diagonal 16x16 blocks (one per warp), then three block levels ---
+  if (warp < 4 && lane < 16) {
+    const int base = 16 * warp, jl = lane;
+    const int bx = base ^ (base & 16);
+    const float* Ab = As + base * 64 + bx;
+    float x[16];
+#pragma unroll
+    for (int tl = 0; tl < 16; ++tl) {
+      float a_row[16];
+#pragma unroll
+      for (int i = 0; i < tl; ++i) a_row[i] = Ab[tl * 64 + (i ^ tl)];
+      float acc0 = (tl == jl) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < tl; i += 2) {
+        acc0 = fmaf(-a_row[i], x[i], acc0);
+        if (i + 1 < tl) acc1 = fmaf(-a_row[i + 1], x[i + 1], acc1);
+      }
+      x[tl] = (tl < jl) ? 0.f : acc0 + acc1;
+    }
+    float* Xb = Xs + base * 64 + bx;
+#pragma unroll
+    for (int tl = 0; tl < 16; ++tl) Xb[tl * 64 + (jl ^ tl)] = x[tl];
+  }
+  __syncthreads();
+  {
+    const int bb = tid >> 6, r = (tid >> 2) & 15, cq = tid & 3;
+#pragma unroll
+    for (int d = 1; d <= 3; ++d) {
+      const bool act = bb < 4 - d;
+      const int aa = bb + d;
+      if (act) {
+        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < d; ++m) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int kk = 16 * (bb + m) + i;
+            const float a = As[sx(16 * aa + r, kk)];
+            float e[4];
+            ld4_sx(Xs, kk, i & 3, 16 * bb + 4 * cq, e);
+            z0 = fmaf(a, e[0], z0);
+            z1 = fmaf(a, e[1], z1);
+            z2 = fmaf(a, e[2], z2);
+            z3 = fmaf(a, e[3], z3);
+          }
+        }
+        *reinterpret_cast<float4*>(&Zs[bb * 256 + r * 16 + 4 * cq]) = make_float4(z0, z1, z2, z3);
+      }
+      __syncthreads();
+      if (act) {
+        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float xa = Xs[sx(16 * aa + r, 16 * aa + i)];
+          const float4 zz = *reinterpret_cast<const float4*>(&Zs[bb * 256 + i * 16 + 4 * cq]);
+          x0 = fmaf(xa, zz.x, x0);
+          x1 = fmaf(xa, zz.y, x1);
+          x2 = fmaf(xa, zz.z, x2);
+          x3 = fmaf(xa, zz.w, x3);
+        }
+        const int row = 16 * aa + r, col = 16 * bb + 4 * cq;
+        Xs[sx(row, col + 0)] = -x0;
+        Xs[sx(row, col + 1)] = -x1;
+        Xs[sx(row, col + 2)] = -x2;
+        Xs[sx(row, col + 3)] = -x3;
+      }
+      __syncthreads();
+    }
+  }
+  // ---- 7. T = X Diag(beta) to the image (blocks above the diagonal are zero) ------------------
+  {
+    const int r = tid & 63, qq = tid >> 6;
+    unsigned char* it = img + WS_T;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      float e[4];
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int j = 16 * qq + 4 * x + y;
+        e[y] = (qq <= (r >> 4)) ? Xs[sx(r, j)] * ps.beta[j] : 0.f;
+      }
+      *reinterpret_cast<float4*>(it + swz_off4(r, 4 * qq + x, 64)) = tf32x4(e[0], e[1], e[2], e[3]);
+    }
+  }
+}
+
+// ========================================================================================
+// Kernel 2: the state carry, per (batch, head, 32-wide slice of d_v)
+// ========================================================================================
+
+constexpr int C_THREADS = 256;               // warps 0-3 carry, warps 4-7 load
+constexpr int C_A = 0;                       // group A image                            64.5 KB
+constexpr int C_C = 66560;                   // T (16 KB) | v bf16 [64 j][32 v] (TMA, 4 KB)
+constexpr int C_V = C_C + 16384;
+constexpr int C_D = C_C + 20480;             // K^ (32 KB) | P (16 KB)
+constexpr int C_SS = C_D + WS_D_BYTES;       // tf32 [32 v][128 c] state operand        16 KB
+constexpr int C_RT = C_SS + 16384;           // tf32 [32 v][64 j] R                       8 KB
+constexpr int C_UT = C_RT + 8192;            // tf32 [32 v][64 j] U                       8 KB
+constexpr int C_OX = C_UT + 8192;            // P U exchange [64 t][32 v] (loader)        8 KB
+constexpr int C_SMALL = C_OX + 8192;
+constexpr int C_SMEM = C_SMALL + 1024 + 1024;
+static_assert(C_C % 1024 == 0 && C_D % 1024 == 0 && C_SS % 1024 == 0, "tile alignment");
+static_assert(C_SMEM <= 232448, "shared memory");
+
+constexpr uint32_t TM_OY = 0;    // [O1; Y] M=128 x 32, + 32 * (c & 1)
+constexpr uint32_t TM_O2 = 64;   // P U, M=64 x 32, + 32 * (c & 1)
+constexpr uint32_t TM_U = 128;   // U, M=64 x 32
+constexpr uint32_t TM_S = 160;   // S^T, M=128 x 32
+constexpr uint32_t C_TM_COLS = 256;
+
+struct CarrySmall {
+  unsigned long long full[3];    // groups A, C, D landed
+  unsigned long long empty[3];   // the products that read groups A, C, D have completed
+  unsigned long long mma_bar;
+  unsigned long long out_full[2];   // chunk's O1 and P U are in TMEM (carry -> loader)
+  unsigned long long out_empty[2];  // loader has read them (loader -> carry)
+  uint32_t tmem;
+  int abort;
+};
+
+template <typename Tout>
+__global__ void __launch_bounds__(C_THREADS, 1)
+kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
+                       const unsigned char* __restrict__ ws, const float* __restrict__ s0,
+                       Tout* __restrict__ o, float* __restrict__ s_final, int T, int H, int dv,
+                       int nchunks, unsigned int* __restrict__ status, uint32_t spin_limit) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sm = smem_raw + padb;
+  CarrySmall& cs = *reinterpret_cast<CarrySmall*>(sm + C_SMALL);
+  unsigned char* tSS = sm + C_SS;
+  unsigned char* tRT = sm + C_RT;
+  unsigned char* tUT = sm + C_UT;
+  float* Ox = reinterpret_cast<float*>(sm + C_OX);
+  uint64_t* full = reinterpret_cast<uint64_t*>(&cs.full[0]);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(&cs.empty[0]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3;
+  const int nslice = dv / kDVS;
+  const int slice = blockIdx.x % nslice;
+  const int bh = blockIdx.x / nslice;
+  const int h = bh % H, b = bh / H;
+  const int v0 = slice * kDVS;
+
+  if (tid == 0) {
+    for (int g = 0; g < 3; ++g) {
+      mbar_init(full + g, 1);
+      mbar_init(empty + g, 1);
+    }
+    mbar_init(reinterpret_cast<uint64_t*>(&cs.mma_bar), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_full[s]), 1);
+      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_empty[s]), 1);
+    }
+    cs.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&cs.tmem, C_TM_COLS);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tb = cs.tmem;
+  const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
+  const unsigned char* wsb = ws + kStatusBytes + (size_t)bh * nchunks * kChunkWs;
+  const uint32_t sbase_u = smem_u32(sm);
+
+  auto give_up = [&](uint64_t* bar, uint32_t parity, bool drain) {
+    if (drain) mbar_wait(bar, parity, kDrainLimit);
+    atomicOr(status, 1u);
+    cs.abort = 1;
+  };
+
+  if (warp >= 4) {
+    // =========================== loader warpgroup =====================================
+    const int lt = tid - 128;
+    auto write_outputs = [&](int cc) -> bool {
+      const int ob = cc & 1;
+      const uint32_t use = (uint32_t)(cc >> 1);
+      uint64_t* ofull = reinterpret_cast<uint64_t*>(&cs.out_full[ob]);
+      if (lt == 0 && !mbar_wait(ofull, use & 1u, spin_limit)) give_up(ofull, use & 1u, false);
+      named_bar(2, 128);
+      if (cs.abort) return false;
+      fence_after_sync();
+      const int t0 = cc * kC;
+      const int L = min(kC, T - t0);
+      {
+        float o2[32];
+        tmem_ld32(tb + tlane + TM_O2 + 32 * ob, o2);
+        tmem_wait_ld();
+        if (lane < 16) {
+          const int t = 16 * q4 + lane;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) Ox[t * 32 + (x ^ (t & 31))] = o2[x];
+        }
+      }
+      named_bar(2, 128);
+      if (q4 < 2) {
+        const int t = 32 * q4 + lane;
+        float o1[32], o2[32];
+        tmem_ld32(tb + tlane + TM_OY + 32 * ob, o1);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
+        tmem_wait_ld();
+        if (t < L) {
+          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
+          if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              uint4 pk;
+              __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                hp[x] = __floats2bfloat162_rn(o1[8 * qq + 2 * x] + o2[8 * qq + 2 * x],
+                                              o1[8 * qq + 2 * x + 1] + o2[8 * qq + 2 * x + 1]);
+              reinterpret_cast<uint4*>(dst)[qq] = pk;
+            }
+          } else {
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq)
+              reinterpret_cast<float4*>(dst)[qq] =
+                  make_float4(o1[4 * qq] + o2[4 * qq], o1[4 * qq + 1] + o2[4 * qq + 1],
+                              o1[4 * qq + 2] + o2[4 * qq + 2], o1[4 * qq + 3] + o2[4 * qq + 3]);
+          }
+        }
+      }
+      fence_before_sync();
+      named_bar(2, 128);
+      if (lt == 0) mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_empty[ob]));
+      return true;
+    };
+    int issued = 0;   // thread lt == 0: groups with a copy in flight or landed, for draining
+    uint32_t last_par = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t par = (uint32_t)c & 1u;
+      if (lt == 0) {
+        // each group: wait until the product that read it for chunk c-1 has completed
+        // (the first use passes at once), then copy chunk c's image in
+        const unsigned char* src = wsb + (size_t)c * kChunkWs;
+        const uint32_t dst[3] = {sbase_u + C_A, sbase_u + C_C, sbase_u + C_D};
+        const uint32_t off[3] = {WS_QK, WS_T, WS_KH};
+        const uint32_t bytes[3] = {WS_A_BYTES, 16384, WS_D_BYTES};
+        issued = 0;
+        last_par = par;
+        for (int g = 0; g < 3; ++g) {
+          if (!mbar_wait(empty + g, par ^ 1u, spin_limit)) {
+            give_up(empty + g, par ^ 1u, false);
+            break;
+          }
+          mbar_expect_tx(full + g, bytes[g] + (g == 1 ? 4096u : 0u));
+          bulk_load(dst[g], src + off[g], bytes[g], full + g);
+          if (g == 1) tma_load_4d(sbase_u + C_V, &tm_v, v0, h, c * kC, b, full + g);
+          issued |= 1 << g;
+        }
+      }
+      named_bar(2, 128);
+      if (cs.abort) break;
+      if (c > 0 && !write_outputs(c - 1)) break;
+    }
+    if (cs.abort && lt == 0) {
+      // copies this thread issued may still be landing in shared memory: let them finish
+      for (int g = 0; g < 3; ++g)
+        if (issued & (1 << g)) mbar_wait(full + g, last_par, kDrainLimit);
+    }
+    if (!cs.abort) write_outputs(nchunks - 1);
+  } else {
+    // =========================== carry warpgroup ======================================
+    const long sbase = ((long)b * H + h) * (long)dv * kDK;
+    float st[kDVS];
+#pragma unroll
+    for (int vv = 0; vv < kDVS; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
+    auto write_state_operand = [&]() {
+#pragma unroll
+      for (int vv = 0; vv < kDVS; ++vv) st_tile(tSS, kDVS, vv, tid, st[vv]);
+    };
+    write_state_operand();
+    fence_smem_to_async();
+    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&cs.mma_bar);
+    uint32_t mphase = 0;
+    const uint64_t dSS = sdesc(smem_u32(tSS), 16, 1024);
+    const uint64_t dRT = sdesc(smem_u32(tRT), 16, 1024), dUT = sdesc(smem_u32(tUT), 16, 1024);
+    const uint64_t dQK = sdesc(sbase_u + C_A, 16, 1024), dT = sdesc(sbase_u + C_C, 16, 1024);
+    const uint64_t dKH = sdesc(sbase_u + C_D, 16, 1024);
+    const uint64_t dP = sdesc(sbase_u + C_D + 32768, 16, 1024);
+    const float* egl = reinterpret_cast<const float*>(sm + C_A + WS_EGL);
+    auto wait_mma = [&]() -> bool {
+      if (!mbar_wait(mma_bar, mphase, spin_limit)) give_up(mma_bar, mphase, true);
+      mphase ^= 1u;
+      fence_after_sync();
+      named_bar(1, 128);
+      return cs.abort != 0;
+    };
+    bool aborted = false;
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t par = (uint32_t)c & 1u;
+      const int ob = c & 1;
+      // ---- group A has landed; the output buffer is free ----------------------------------
+      if (tid == 0) {
+        if (!mbar_wait(full + 0, par, spin_limit)) give_up(full + 0, par, true);
+        if (c >= 2) {
+          uint64_t* oe = reinterpret_cast<uint64_t*>(&cs.out_empty[ob]);
+          const uint32_t p2 = (uint32_t)((c >> 1) - 1) & 1u;
+          if (!mbar_wait(oe, p2, spin_limit)) give_up(oe, p2, false);
+        }
+      }
+      named_bar(1, 128);
+      if ((aborted = cs.abort != 0)) break;
+      fence_after_sync();
+      // ---- decay the state in TMEM, then [O1; Y] = [Q~; K~] S0^T -----------------------------
+      {
+        float sd[kDVS];
+        const float e = egl[tid];
+#pragma unroll
+        for (int vv = 0; vv < kDVS; ++vv) sd[vv] = st[vv] * e;
+        tmem_st32(tb + tlane + TM_S, sd);
+        tmem_wait_st();
+      }
+      fence_before_sync();
+      named_bar(1, 128);
+      if (tid == 0) {
+        fence_after_sync();
+        const uint32_t id = idesc_tf32(128, 32, false, false);
+#pragma unroll 4
+        for (int ks = 0; ks < kDK / 8; ++ks)
+          mma_tf32(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSS, kDVS, ks), id, ks > 0);
+        mma_commit(mma_bar);
+        mma_commit(empty + 0);
+        if (!mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
+      }
+      if ((aborted = wait_mma())) break;
+      // ---- R = V - Y as the operand [v][j] (Y rows: TMEM lanes 64-127) ------------------------
+      if (q4 >= 2) {
+        const int j = 32 * (q4 - 2) + lane;
+        float y[32], vv[32];
+        const uint4* vrow = reinterpret_cast<const uint4*>(sm + C_V + j * 64);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint4 raw = vrow[qq];
+          const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float2 f = __bfloat1622float2(hh[x]);
+            vv[8 * qq + 2 * x] = f.x;
+            vv[8 * qq + 2 * x + 1] = f.y;
+          }
+        }
+        tmem_ld32(tb + tlane + TM_OY + 32 * ob, y);
+        tmem_wait_ld();
+#pragma unroll
+        for (int v = 0; v < kDVS; ++v) st_tile(tRT, kDVS, v, j, vv[v] - y[v]);
+      }
+      fence_smem_to_async();
+      fence_before_sync();
+      named_bar(1, 128);
+      // ---- U = T R ---------------------------------------------------------------------------
+      if (tid == 0) {
+        fence_after_sync();
+        const uint32_t id = idesc_tf32(64, 32, false, false);
+#pragma unroll
+        for (int ks = 0; ks < kC / 8; ++ks)
+          mma_tf32(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
+        mma_commit(mma_bar);
+        mma_commit(empty + 1);
+        if (!mbar_wait(full + 2, par, spin_limit)) give_up(full + 2, par, true);
+      }
+      if ((aborted = wait_mma())) break;
+      {
+        float u[32];
+        tmem_ld32(tb + tlane + TM_U, u);
+        tmem_wait_ld();
+        if (lane < 16) {
+          const int j = 16 * q4 + lane;
+#pragma unroll
+          for (int v = 0; v < kDVS; ++v) st_tile(tUT, kDVS, v, j, u[v]);
+        }
+      }
+      fence_smem_to_async();
+      fence_before_sync();
+      named_bar(1, 128);
+      // ---- O2 = P U;  S^T += K^ U ------------------------------------------------------------
+      if (tid == 0) {
+        fence_after_sync();
+        const uint32_t i64 = idesc_tf32(64, 32, false, false);
+        const uint32_t i128 = idesc_tf32(128, 32, false, false);
+#pragma unroll
+        for (int ks = 0; ks < kC / 8; ++ks)
+          mma_tf32(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), i64, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < kC / 8; ++ks)
+          mma_tf32(tb + TM_S, kstep(dKH, 128, ks), kstep(dUT, kDVS, ks), i128, true);
+        mma_commit(mma_bar);
+        mma_commit(empty + 2);
+        mma_commit(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
+      }
+      if ((aborted = wait_mma())) break;
+      // ---- new state ---------------------------------------------------------------------------
+      tmem_ld32(tb + tlane + TM_S, st);
+      tmem_wait_ld();
+      write_state_operand();
+      fence_smem_to_async();
+      fence_before_sync();
+      named_bar(1, 128);
+    }
+    if (!aborted && s_final) {
+#pragma unroll
+      for (int vv = 0; vv < kDVS; ++vv) s_final[sbase + (long)(v0 + vv) * kDK + tid] = st[vv];
+    }
+    if (aborted) cs.abort = 1;
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, C_TM_COLS);
+}
+
+uint32_t kda_split_spin_limit() {
+  const char* e = getenv("GDR_SPIN_LIMIT");
+  if (!e || !*e) return 1u << 24;
+  return (uint32_t)strtoul(e, nullptr, 10);
+}
+
+template <typename Tout>
+cudaError_t launch_kda_split_t(const PrefillArgs& a, cudaStream_t stream) {
+  CUtensorMap mv;
+  if (!encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC, false))
+    return cudaErrorInvalidValue;
+  const int nchunks = (a.T + kC - 1) / kC;
+  const uint32_t lim = kda_split_spin_limit();
+  cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (e != cudaSuccess) return e;
+  kda_chunk_prep_kernel<<<a.B * a.H * nchunks, P_THREADS, P_SMEM, stream>>>(
+      (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.alpha, a.beta,
+      (unsigned char*)a.workspace, a.T, a.H, nchunks, (unsigned int*)a.workspace, lim);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto carry = kda_chunk_carry_kernel<Tout>;
+  e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
+  if (e != cudaSuccess) return e;
+  carry<<<a.B * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
+      mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, a.T, a.H, a.dv, nchunks,
+      (unsigned int*)a.workspace, lim);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t kda_split_workspace(int B, int T, int H) {
+  const size_t nchunks = ((size_t)T + kC - 1) / kC;
+  return (size_t)B * H * nchunks * kChunkWs;
+}
+
+cudaError_t launch_prefill_kda_split(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.out_dtype == GDR_F32) return launch_kda_split_t<float>(a, stream);
+  return launch_kda_split_t<__nv_bfloat16>(a, stream);
+}
+
+}  // namespace gdr

@@ -621,20 +621,27 @@ bool tc_prefill_supported(const PrefillArgs& a) {
 size_t split_prefill_workspace(int B, int T, int H);            // prefill_split.cu
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_kda_tc(const PrefillArgs& a, cudaStream_t stream);  // prefill_kda_tc.cu
+size_t kda_split_workspace(int B, int T, int H);                                // prefill_kda_split.cu
+cudaError_t launch_prefill_kda_split(const PrefillArgs& a, cudaStream_t stream);
 
-// The two-kernel path (per-chunk prep over the whole GPU, then the carry) needs a
-// workspace of 33 KB per chunk; with a smaller workspace this single-kernel path runs.
+// The two-kernel paths (per-chunk prep over the whole GPU, then the carry) need a
+// workspace of 33 KB (GDN) or 128.5 KB (KDA) per chunk; with a smaller workspace the
+// single-kernel kernels run.
 size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
   PrefillArgs a{};
   a.in_dtype = GDR_BF16;
   a.dk = dk;
   a.dv = dv;
   a.kda = kda;
-  return tc_prefill_supported(a) && !kda ? split_prefill_workspace(B, T, H) : 0;
+  if (!tc_prefill_supported(a)) return 0;
+  return kda ? kda_split_workspace(B, T, H) : split_prefill_workspace(B, T, H);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
-  if (a.kda) return launch_prefill_kda_tc(a, st);
+  if (a.kda) {
+    if (a.ws_bytes >= 256 + kda_split_workspace(a.B, a.T, a.H)) return launch_prefill_kda_split(a, st);
+    return launch_prefill_kda_tc(a, st);
+  }
   if (a.ws_bytes >= 256 + split_prefill_workspace(a.B, a.T, a.H)) return launch_prefill_split(a, st);
   if (a.out_dtype == GDR_F32) return launch_t<float>(a, st);
   return launch_t<__nv_bfloat16>(a, st);

@@ -14,18 +14,21 @@ from synth import Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("mixer", ["gdn", "kda"])
 @pytest.mark.parametrize("path", ["single-kernel", "two-kernel"])
-def test_bounded_wait_reports_timeout_and_recovers(path):
+def test_bounded_wait_reports_timeout_and_recovers(mixer, path):
     import gated_delta_rule_79_b200 as g
-    w = Workload("fi", "gdn", 1, 2, 100, 128, 128, "bf16", "randn")
+    kda = mixer == "kda"
+    w = Workload("fi", mixer, 1, 2, 100, 128, 128, "bf16", "randn")
     x = {k: v.cuda() for k, v in make_inputs(w, seed=11).items()}
-    assert g.prefill_path(128, 128, torch.bfloat16, False) == "tensor-core"
-    full = g.lib.gdr_prefill_workspace_bytes(1, 100, 2, 128, 128, 0)
+    assert g.prefill_path(128, 128, torch.bfloat16, kda) == "tensor-core"
+    fn = g.kda_prefill if kda else g.gdn_prefill
+    full = g.lib.gdr_prefill_workspace_bytes(1, 100, 2, 128, 128, int(kda))
     ws = torch.zeros(4096 if path == "single-kernel" else full, dtype=torch.uint8, device="cuda")
     old = os.environ.get("GDR_SPIN_LIMIT")
     os.environ["GDR_SPIN_LIMIT"] = "0"
     try:
-        g.gdn_prefill(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], workspace=ws)
+        fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], workspace=ws)
         with pytest.raises(g.GdrError) as e:
             g.workspace_status(ws)
         assert e.value.status == g.GDR_ERR_TIMEOUT
@@ -35,6 +38,6 @@ def test_bounded_wait_reports_timeout_and_recovers(path):
         else:
             os.environ["GDR_SPIN_LIMIT"] = old
     # the status word was cleared and the context is healthy
-    o, s = g.gdn_prefill(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], workspace=ws)
+    o, s = fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], workspace=ws)
     g.workspace_status(ws)
     assert torch.isfinite(o.float()).all() and torch.isfinite(s).all()

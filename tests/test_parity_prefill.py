@@ -18,11 +18,12 @@ pytestmark = pytest.mark.gpu
 TOL = {"f32": 1e-5, "bf16": 2e-3}
 
 
-def gpu_prefill(mixer, x, out_dtype=None):
+def gpu_prefill(mixer, x, out_dtype=None, workspace=None):
     import gated_delta_rule_79_b200 as g
     fn = g.kda_prefill if mixer == "kda" else g.gdn_prefill
     t = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
-    o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], t["s0"], out_dtype=out_dtype)
+    o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], t["s0"], out_dtype=out_dtype,
+              workspace=workspace)
     torch.cuda.synchronize()
     return to_np(o), to_np(s)
 
@@ -76,6 +77,22 @@ def test_stress_gates(mixer, dtype, gates):
     o, s = gpu_prefill(mixer, x, out_dtype=torch.float32)
     o_ref, s_ref = ref_prefill(x)
     check(o, s, o_ref, s_ref, TOL[dtype], f"{mixer} {dtype} gates={gates}")
+
+
+@pytest.mark.parametrize("mixer", ["gdn", "kda"])
+@pytest.mark.parametrize("gates", ["workload", "slow", "zero_some"])
+@pytest.mark.parametrize("T", [77, 200])
+def test_single_kernel_path(mixer, gates, T):
+    """With a workspace that holds only the status word, bf16 d=128 prefill runs the
+    single-kernel tensor-core kernels instead of the two-kernel ones."""
+    import gated_delta_rule_79_b200 as g
+    w = Workload("single", mixer, 2, 2, T, 128, 128, "bf16", "randn")
+    x = make_inputs(w, seed=T + 3, gates=gates)
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    o, s = gpu_prefill(mixer, x, out_dtype=torch.float32, workspace=ws)
+    g.workspace_status(ws)
+    o_ref, s_ref = ref_prefill(x)
+    check(o, s, o_ref, s_ref, TOL["bf16"], f"single-kernel {mixer} gates={gates} T={T}")
 
 
 @pytest.mark.parametrize("T", [63, 64, 127, 128, 129])
