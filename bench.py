@@ -73,8 +73,8 @@ def load_peaks():
 
 
 def load_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current source of the kernel (else None)."""
+    """DRAM bytes per call from the committed ncu summary, if it was taken on the
+    current source of the kernels (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -90,11 +90,17 @@ def load_traffic(kernel_key):
 
 
 def source_sha(rel):
+    """First 16 hex digits of the sha256 of a source file, or of several files'
+    contents concatenated (rel a list)."""
     import hashlib
-    p = os.path.join(ROOT, rel)
-    if not rel or not os.path.exists(p):
-        return None
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    rels = rel if isinstance(rel, list) else [rel]
+    h = hashlib.sha256()
+    for r in rels:
+        p = os.path.join(ROOT, r)
+        if not r or not os.path.exists(p):
+            return None
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
 
 
 # ----------------------------------------------------------------------------------------
@@ -210,8 +216,16 @@ class PrefillRunner:
         self.s = [torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
                   for _ in self.sets]
         self.ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev)
-        self.launches_per_step = 1
         self.path = g.prefill_path(w.dk, w.dv, w.torch_dtype, w.mixer == "kda")
+        # the tensor-core path with a full-size workspace runs a per-chunk prep kernel,
+        # then the state carry; the others run one kernel per call
+        if self.path == "tensor-core":
+            self.kernels = [f"{w.mixer}_chunk_prep_kernel", f"{w.mixer}_chunk_carry_kernel"]
+            self.kernel_key = f"prefill_two-kernel:{w.name}"
+        else:
+            self.kernels = ["prefill_simt_kernel"]
+            self.kernel_key = f"prefill_{self.path}:{w.name}"
+        self.launches_per_step = len(self.kernels)
         self.l2_note = f"{len(self.sets)} rotating input sets of {set_bytes / 2**20:.0f} MiB (> 3x L2)"
 
     def step(self, i):
@@ -232,6 +246,8 @@ class DecodeRunner:
         self.state = self.x["s0"]
         self.o = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
         self.launches_per_step = w.T
+        self.kernels = ["decode_kernel"]
+        self.kernel_key = f"decode:{w.name}"
         self.path = "decode (CUDA cores, fp32 state)"
         self.l2_note = f"state of {self.state.numel() * 4 / 2**20:.0f} MiB > L2"
 
@@ -245,7 +261,9 @@ class DecodeRunner:
 def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
     """Warm up, then time exactly `steps` steps with CUDA events on the launching
     stream, bracketed by a barrier and a synchronize on both sides.  Also records
-    each step's own event pair (the kernel-duration evidence for the roofline)."""
+    each step's own event pair (the kernel-duration evidence for the roofline) and,
+    for prefill, the library's per-kernel events on the same stream (the mean
+    duration of each kernel of a call)."""
     stream = torch.cuda.current_stream(dev)
     for i in range(warmup):
         runner.step(i)
@@ -264,6 +282,9 @@ def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
           for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    per_kernel = not runner.w.decode
+    if per_kernel:
+        runner.g.timing_start()
     t0.record(stream)
     for i in range(steps):
         ev[i][0].record(stream)
@@ -271,10 +292,11 @@ def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
         ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    kernel_ms = runner.g.timing_stop()[0] if per_kernel else None
     barrier(active, dev)
     total_ms = t0.elapsed_time(t1)
     per = [a.elapsed_time(b) for a, b in ev]
-    return total_ms, per
+    return total_ms, per, kernel_ms
 
 
 def time_e2e(w, dev, steps, warmup, seed):
@@ -438,7 +460,7 @@ def main():
     runner = (DecodeRunner if w.decode else PrefillRunner)(w, dev, seed=1000 * rank)
     clocks = ClockSampler(dev.index)
     clocks.start()
-    total_ms, per = time_device(runner, steps, warmup, dev, active)
+    total_ms, per, kernel_ms = time_device(runner, steps, warmup, dev, active)
     clk = clocks.stop()
     ms_step = total_ms / steps
     max_ms = max_over_ranks(total_ms, active, dev)
@@ -456,12 +478,20 @@ def main():
         launch_ms, bytes_launch, flops_launch = kern_ms, nbytes, flops
     hbm = bytes_launch / (launch_ms / 1e3) / 1e9
     tflops = flops_launch / (launch_ms / 1e3) / 1e12
-    kernel_key = ("decode" if w.decode else f"prefill_{runner.path}") + f":{w.name}"
-    traffic = load_traffic(kernel_key)
+    traffic = load_traffic(runner.kernel_key)
     roofline = {"bound": "hbm", "achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": hbm / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
                 "launch_ms": launch_ms}
+    if kernel_ms:
+        # one "launch" of the roofline is one call of the path; its kernels, timed
+        # with events on the launching stream over the same timed steps:
+        tot = sum(kernel_ms)
+        roofline["launch"] = "one prefill call (" + " + ".join(runner.kernels) + ")"
+        roofline["kernels"] = [{"name": n, "ms": m, "share": m / tot if tot else None}
+                               for n, m in zip(runner.kernels, kernel_ms)]
+        dom = max(range(len(kernel_ms)), key=lambda i: kernel_ms[i])
+        roofline["dominant"] = runner.kernels[dom] if dom < len(runner.kernels) else None
     extra = {}
     if not w.decode:
         extra["roofline_tensor"] = {

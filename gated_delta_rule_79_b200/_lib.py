@@ -22,7 +22,7 @@ CHUNK = 64
 
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
-           "gdr_prefill_path", "gdn_prefill_noalloc"]
+           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop"]
 
 
 class GdrError(RuntimeError):
@@ -58,6 +58,10 @@ def _load():
     lib.gdr_prefill_path.argtypes = [i, i, i, i]
     lib.gdr_workspace_status.restype = i
     lib.gdr_workspace_status.argtypes = [vp, sz, vp]
+    lib.gdr_timing_start.restype = i
+    lib.gdr_timing_start.argtypes = []
+    lib.gdr_timing_stop.restype = i
+    lib.gdr_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_float), i, ctypes.POINTER(i)]
     return lib
 
 
@@ -225,3 +229,18 @@ def workspace_status(workspace, stream=None):
     raises GdrError(GDR_ERR_TIMEOUT) if a bounded device wait gave up."""
     dev = workspace.device
     _check(lib.gdr_workspace_status(_ptr(workspace), workspace.numel(), _stream(dev, stream)))
+
+
+def timing_start():
+    """Start recording per-kernel CUDA events for every prefill call (measurement aid)."""
+    lib.gdr_timing_start()
+
+
+def timing_stop(max_kernels=8):
+    """Stop recording; returns (mean ms of each kernel position of a call, calls)."""
+    buf = (ctypes.c_float * max_kernels)()
+    n = ctypes.c_int(0)
+    k = lib.gdr_timing_stop(buf, max_kernels, ctypes.byref(n))
+    if k < 0:
+        raise GdrError(GDR_ERR_CUDA, "gdr_timing_stop: reading a CUDA event failed")
+    return [float(buf[i]) for i in range(min(k, max_kernels))], int(n.value)

@@ -90,6 +90,7 @@ static gdr_status prefill(bool kda, const void* q, const void* k, const void* v,
     return fail(GDR_ERR_INVALID_ARG, "%s: s0/s_final not 16-byte aligned", fn);
   PrefillArgs a{q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv,
                 in_dtype, out_dtype, kda, workspace, ws_bytes};
+  timing_mark(st, -1);
   cudaError_t e = tc_prefill_supported(a) ? launch_prefill_tc(a, st) : launch_prefill_simt(a, st);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return ok();

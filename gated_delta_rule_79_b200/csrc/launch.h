@@ -39,6 +39,10 @@ struct DecodeArgs {
 // Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
 int report_error(int s, const char* msg);
 
+// Measurement aid (timing.cu): records an event on `stream` when timing is on.
+// slot -1 marks the start of a prefill call, slot i the end of its i-th kernel.
+void timing_mark(cudaStream_t stream, int slot);
+
 // Each returns cudaSuccess or the launch error; messages are set by the caller.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);

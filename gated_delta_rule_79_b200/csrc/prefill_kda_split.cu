@@ -112,12 +112,15 @@ struct PrepSmall {
   unsigned wmask[4];    // wide channels
   uint32_t tmem;
   unsigned long long mma_bar;
+  unsigned long long tma_bar;
 };
 static_assert(sizeof(PrepSmall) <= 3072, "prep small");
 
 __global__ void __launch_bounds__(P_THREADS, 2)
-kda_chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                      const float* __restrict__ alpha, const float* __restrict__ beta,
+kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_a, const __nv_bfloat16* __restrict__ q,
+                      const __nv_bfloat16* __restrict__ k, const float* __restrict__ beta,
                       unsigned char* __restrict__ ws, int T, int H, int nchunks,
                       unsigned int* __restrict__ status, uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
@@ -131,6 +134,7 @@ kda_chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   float* Gw = reinterpret_cast<float*>(tR);
   PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(&ps.tma_bar);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, hw = warp >> 2;
@@ -142,56 +146,62 @@ kda_chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   const long row0 = ((long)b * T + t0) * H + h;    // token t of the chunk: row0 + t * H
   unsigned char* img = ws + kStatusBytes + ((size_t)bh * nchunks + c) * kChunkWs;
 
+  // the chunk's q and k (bf16 [64 t][128 c]) land in the L area and its gates (fp32
+  // [64 t][128 c]) in the R area; both are read into registers before L and R are built
   if (tid == 0) {
     mbar_init(mma_bar, 1);
+    mbar_init(tma_bar, 1);
     fence_mbar_init();
+    mbar_expect_tx(tma_bar, 16384 + 16384 + 32768);
+    tma_load_4d(smem_u32(tL), &tm_q, 0, h, t0, b, tma_bar);
+    tma_load_4d(smem_u32(tL) + 16384, &tm_k, 0, h, t0, b, tma_bar);
+    tma_load_4d(smem_u32(tR), &tm_a, 0, h, t0, b, tma_bar);
   }
   if (warp == 0) tmem_alloc(&ps.tmem, P_TM_COLS);
-  // ---- 1. this thread's channel cc, tokens 32 hw .. 32 hw + 31 (rows past T: alpha 1, 0)
+  if (tid < kC) ps.beta[tid] = tid < L ? beta[row0 + (long)tid * H] : 0.f;
+  fence_before_sync();
+  __syncthreads();
+  // ---- 1. this thread's channel cc, tokens 32 hw .. 32 hw + 31 (rows past T read as 0)
   const int cc = 32 * q4 + lane;
   float g[32];
   uint32_t qp[16], kp[16];   // bf16 pairs: tokens (2i, 2i+1) of the half
   {
-    const unsigned short* qs = reinterpret_cast<const unsigned short*>(q);
-    const unsigned short* ks = reinterpret_cast<const unsigned short*>(k);
+    bool failed = false;
+    if (!mbar_wait(tma_bar, 0, spin_limit)) {
+      mbar_wait(tma_bar, 0, kDrainLimit);
+      failed = true;
+    }
+    if (__syncthreads_or(failed)) {
+      if (lane == 0) atomicOr(status, 1u);
+      fence_after_sync();
+      if (warp == 0) tmem_dealloc(ps.tmem, P_TM_COLS);
+      return;
+    }
+    const unsigned short* qs = reinterpret_cast<const unsigned short*>(tL);
+    const unsigned short* ks = reinterpret_cast<const unsigned short*>(tL + 16384);
+    const float* as = reinterpret_cast<const float*>(tR);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      uint32_t qa = 0, qb = 0, ka = 0, kb = 0;
-      const int ta = 32 * hw + 2 * i, tb2 = ta + 1;
-      if (ta < L) {
-        const long e = (row0 + (long)ta * H) * kDK + cc;
-        g[2 * i] = __ldg(alpha + e);
-        qa = __ldg(qs + e);
-        ka = __ldg(ks + e);
-      } else {
-        g[2 * i] = 1.f;
-      }
-      if (tb2 < L) {
-        const long e = (row0 + (long)tb2 * H) * kDK + cc;
-        g[2 * i + 1] = __ldg(alpha + e);
-        qb = __ldg(qs + e);
-        kb = __ldg(ks + e);
-      } else {
-        g[2 * i + 1] = 1.f;
-      }
-      qp[i] = qa | (qb << 16);
-      kp[i] = ka | (kb << 16);
+      const int ta = 32 * hw + 2 * i;
+      qp[i] = (uint32_t)qs[ta * kDK + cc] | ((uint32_t)qs[(ta + 1) * kDK + cc] << 16);
+      kp[i] = (uint32_t)ks[ta * kDK + cc] | ((uint32_t)ks[(ta + 1) * kDK + cc] << 16);
+      g[2 * i] = as[ta * kDK + cc];
+      g[2 * i + 1] = as[(ta + 1) * kDK + cc];
     }
   }
-  if (tid < kC) ps.beta[tid] = tid < L ? beta[row0 + (long)tid * H] : 0.f;
   // ---- 2. cumulative log gate: fp64 prefix over each half, halves joined by their sums
   {
     double acc = 0.0;
 #pragma unroll
     for (int x = 0; x < 32; ++x) {
-      acc += (double)log_gate_accurate(g[x]);
+      acc += (32 * hw + x < L) ? (double)log_gate(g[x]) : 0.0;
       g[x] = (float)acc;
     }
     ps.tot[hw][cc] = acc;
     if (hw == 0) ps.g0[cc] = g[0];
   }
   fence_before_sync();
-  __syncthreads();
+  __syncthreads();   // also: every read of the staged q, k and gates is done
   fence_after_sync();
   const uint32_t tb = ps.tmem;
   const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
@@ -751,8 +761,11 @@ uint32_t kda_split_spin_limit() {
 
 template <typename Tout>
 cudaError_t launch_kda_split_t(const PrefillArgs& a, cudaStream_t stream) {
-  CUtensorMap mv;
-  if (!encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC, false))
+  CUtensorMap mq, mk, ma, mv;
+  if (!encode_bthd_bf16(&mq, a.q, a.B, a.T, a.H, kDK, kDK, kC, false) ||
+      !encode_bthd_bf16(&mk, a.k, a.B, a.T, a.H, kDK, kDK, kC, false) ||
+      !encode_bthd_f32(&ma, a.alpha, a.B, a.T, a.H, kDK, kDK, kC) ||
+      !encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC, false))
     return cudaErrorInvalidValue;
   const int nchunks = (a.T + kC - 1) / kC;
   const uint32_t lim = kda_split_spin_limit();
@@ -760,17 +773,20 @@ cudaError_t launch_kda_split_t(const PrefillArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
   kda_chunk_prep_kernel<<<a.B * a.H * nchunks, P_THREADS, P_SMEM, stream>>>(
-      (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.alpha, a.beta,
+      mq, mk, ma, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.beta,
       (unsigned char*)a.workspace, a.T, a.H, nchunks, (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  timing_mark(stream, 0);
   auto carry = kda_chunk_carry_kernel<Tout>;
   e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return e;
   carry<<<a.B * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
       mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, a.T, a.H, a.dv, nchunks,
       (unsigned int*)a.workspace, lim);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) timing_mark(stream, 1);
+  return e;
 }
 
 }  // namespace

@@ -582,27 +582,13 @@ uint32_t kda_spin_limit() {
   return (uint32_t)strtoul(e, nullptr, 10);
 }
 
-// Tensor map over the fp32 per-channel gates [B, T, H, 128]: boxes of 128 channels x 64
-// tokens; rows past T read as zero (the kernel treats them as alpha = 1).
-bool encode_gates(CUtensorMap* m, const float* base, int B, int T, int H) {
-  auto fn = tensor_map_encoder();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)kDK, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)kDK * 4, (cuuint64_t)H * kDK * 4, (cuuint64_t)T * H * kDK * 4};
-  cuuint32_t box[4] = {(cuuint32_t)kDK, 1, (cuuint32_t)kC, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename Tout>
 cudaError_t launch_kda_t(const PrefillArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, ma;
   if (!encode_bthd_bf16(&mq, a.q, a.B, a.T, a.H, kDK, kDK, kC) ||
       !encode_bthd_bf16(&mk, a.k, a.B, a.T, a.H, kDK, kDK, kC) ||
       !encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC) ||
-      !encode_gates(&ma, a.alpha, a.B, a.T, a.H))
+      !encode_bthd_f32(&ma, a.alpha, a.B, a.T, a.H, kDK, kDK, kC))
     return cudaErrorInvalidValue;
   auto kern = kda_prefill_tc_kernel<Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -610,7 +596,9 @@ cudaError_t launch_kda_t(const PrefillArgs& a, cudaStream_t st) {
   kern<<<a.B * a.H * (a.dv / kDVS), kThreads, SMEM_BYTES, st>>>(
       mq, mk, mv, ma, a.beta, a.s0, (Tout*)a.o, a.s_final, a.T, a.H, a.dv,
       (unsigned int*)a.workspace, kda_spin_limit());
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) timing_mark(st, 0);
+  return e;
 }
 
 }  // namespace

@@ -265,7 +265,9 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st) {
   kern<<<grid, kThreads, L::BYTES, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                          a.alpha, a.beta, a.s0, (Tout*)a.o, a.s_final,
                                          a.T, a.H, a.dv);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) timing_mark(st, 0);
+  return e;
 }
 
 template <int DK, bool KDA>

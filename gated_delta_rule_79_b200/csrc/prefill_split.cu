@@ -780,13 +780,16 @@ cudaError_t launch_split_t(const PrefillArgs& a, cudaStream_t stream) {
       (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  timing_mark(stream, 0);
   auto carry = gdn_chunk_carry_kernel<Tout>;
   e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return e;
   carry<<<a.B * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
       mq, mk, mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, a.T, a.H,
       a.dv, nchunks, (unsigned int*)a.workspace, lim);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) timing_mark(stream, 1);
+  return e;
 }
 
 }  // namespace

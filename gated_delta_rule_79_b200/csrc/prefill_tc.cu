@@ -607,7 +607,9 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st) {
   kern<<<grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mv, a.alpha, a.beta, a.s0, (Tout*)a.o,
                                            a.s_final, a.T, a.H, a.dv, (unsigned int*)a.workspace,
                                            spin_limit_from_env());
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) timing_mark(st, 0);
+  return e;
 }
 
 }  // namespace

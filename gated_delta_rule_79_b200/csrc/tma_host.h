@@ -43,4 +43,21 @@ inline bool encode_bthd_bf16(CUtensorMap* m, const void* base, int B, int T, int
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a dense fp32 tensor [B, T, H, D] (D contiguous, D * 4 a multiple of
+// 16 bytes) with boxes of `box_d` x 1 head x `box_t` tokens x 1 batch, no swizzle;
+// rows past T read as zero.
+inline bool encode_bthd_f32(CUtensorMap* m, const float* base, int B, int T, int H, int D,
+                            int box_d, int box_t) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+  cuuint32_t box[4] = {(cuuint32_t)box_d, 1, (cuuint32_t)box_t, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace gdr

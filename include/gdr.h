@@ -170,6 +170,18 @@ GDR_API int gdr_prefill_path(int dk, int dv, int in_dtype, int kda);
  * then undefined), or GDR_ERR_CUDA. */
 GDR_API gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream);
 
+/* Measurement aid; the paper has no counterpart.  gdr_timing_start() clears the
+ * record and makes every later prefill call record a CUDA event on its stream when
+ * it starts and after each kernel it launches (the two-kernel paths launch a
+ * per-chunk prep kernel, then the state carry).  gdr_timing_stop() stops
+ * recording, waits for the recorded events and writes to avg_ms[i] the mean
+ * duration in milliseconds of the i-th kernel of a call over the recorded calls
+ * (at most max_kernels entries; avg_ms may be NULL), and the number of recorded
+ * calls to *ncalls (may be NULL).  Returns the number of kernels per call, or -1
+ * if reading an event failed.  Process-wide; not for use inside stream capture. */
+GDR_API int gdr_timing_start(void);
+GDR_API int gdr_timing_stop(float* avg_ms, int max_kernels, int* ncalls);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -95,3 +95,10 @@ def test_decode_rejects_bad_arguments(g, fn):
     assert call(alpha=P + 4) == g.GDR_ERR_INVALID_ARG
     assert call(oo=3) == g.GDR_ERR_INVALID_ARG
     assert call(N=0) == g.GDR_OK
+
+
+def test_public_names_resolve():
+    """Every name the package advertises resolves to the binding."""
+    import gated_delta_rule_79_b200 as g
+    for name in g.__all__:
+        assert getattr(g, name) is not None, name
