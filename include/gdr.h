@@ -77,10 +77,11 @@ GDR_API const char* gdr_last_error(void);
 /* Bytes of device workspace with which gdn_prefill / kda_prefill run their
  * fastest path for these sizes (kda != 0 selects KDA); 0 when the sizes are
  * invalid.  The workspace holds the device status word of the bounded waits
- * (the first 256 bytes) and, for the bf16 GDN two-kernel prefill, 33 KB per
- * chunk of 64 tokens per (sequence, head) of precomputed chunk operands.  Any
- * workspace of at least 256 bytes is accepted: with less than the returned size
- * the single-kernel path runs.  It must be zero-filled once when allocated; the
+ * (the first 256 bytes) and, for the bf16 two-kernel prefills (d_k = 128, d_v a
+ * multiple of 32), the precomputed operands of every chunk of 64 tokens per
+ * (sequence, head): 33 KB for GDN, 128.5 KB for KDA.  Any workspace of at least
+ * 256 bytes is accepted: with less than the returned size the single-kernel
+ * tensor-core path runs (slower; it needs the status word only).  It must be zero-filled once when allocated; the
  * library leaves it ready for the next call. */
 GDR_API size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, int kda);
 
