@@ -240,13 +240,13 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   fence_after_sync();
   const bool anywide = (ps.wmask[0] | ps.wmask[1] | ps.wmask[2] | ps.wmask[3]) != 0u;
-  if (tid == 0) {
+  if (warp == 0) {
     const uint64_t dL = sdesc(smem_u32(tL), 16, 1024), dR = sdesc(smem_u32(tR), 16, 1024);
     const uint32_t id = idesc_tf32(128, 64, false, false);
-#pragma unroll 4
+#pragma unroll
     for (int ks = 0; ks < kDK / 8; ++ks)
-      mma_tf32(tb + P_TM_G, kstep(dL, 128, ks), kstep(dR, 64, ks), id, ks > 0);
-    mma_commit(mma_bar);
+      mma_tf32_w(tb + P_TM_G, kstep(dL, 128, ks), kstep(dR, 64, ks), id, ks > 0);
+    mma_commit_w(mma_bar);
   }
   // ---- 4. while the Gram runs: the carry's [Q~; K~], e^{G_last} and K^ images -------------
   {
@@ -658,15 +658,16 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       }
       fence_before_sync();
       named_bar(1, 128);
-      if (tid == 0) {
+      if (warp == 0) {
         fence_after_sync();
         const uint32_t id = idesc_tf32(128, 32, false, false);
-#pragma unroll 4
+#pragma unroll
         for (int ks = 0; ks < kDK / 8; ++ks)
-          mma_tf32(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSS, kDVS, ks), id, ks > 0);
-        mma_commit(mma_bar);
-        mma_commit(empty + 0);
-        if (!mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
+          mma_tf32_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSS, kDVS, ks), id, ks > 0);
+        mma_commit_w(mma_bar);
+        mma_commit_w(empty + 0);
+        if (lane == 0 && !mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
+        __syncwarp();
       }
       if ((aborted = wait_mma())) break;
       // ---- R = V - Y as the operand [v][j] (Y rows: TMEM lanes 64-127) ------------------------
@@ -694,15 +695,16 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       fence_before_sync();
       named_bar(1, 128);
       // ---- U = T R ---------------------------------------------------------------------------
-      if (tid == 0) {
+      if (warp == 0) {
         fence_after_sync();
         const uint32_t id = idesc_tf32(64, 32, false, false);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
-        mma_commit(mma_bar);
-        mma_commit(empty + 1);
-        if (!mbar_wait(full + 2, par, spin_limit)) give_up(full + 2, par, true);
+          mma_tf32_w(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
+        mma_commit_w(mma_bar);
+        mma_commit_w(empty + 1);
+        if (lane == 0 && !mbar_wait(full + 2, par, spin_limit)) give_up(full + 2, par, true);
+        __syncwarp();
       }
       if ((aborted = wait_mma())) break;
       {
@@ -719,19 +721,21 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       fence_before_sync();
       named_bar(1, 128);
       // ---- O2 = P U;  S^T += K^ U ------------------------------------------------------------
-      if (tid == 0) {
+      if (warp == 0) {
+        // the state update first: the chain continues as soon as it completes, while
+        // P U (needed only for the outputs) runs behind it
         fence_after_sync();
         const uint32_t i64 = idesc_tf32(64, 32, false, false);
         const uint32_t i128 = idesc_tf32(128, 32, false, false);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), i64, ks > 0);
+          mma_tf32_w(tb + TM_S, kstep(dKH, 128, ks), kstep(dUT, kDVS, ks), i128, true);
+        mma_commit_w(mma_bar);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_S, kstep(dKH, 128, ks), kstep(dUT, kDVS, ks), i128, true);
-        mma_commit(mma_bar);
-        mma_commit(empty + 2);
-        mma_commit(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
+          mma_tf32_w(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), i64, ks > 0);
+        mma_commit_w(empty + 2);
+        mma_commit_w(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
       }
       if ((aborted = wait_mma())) break;
       // ---- new state ---------------------------------------------------------------------------

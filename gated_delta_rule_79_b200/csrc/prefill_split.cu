@@ -188,15 +188,14 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
     return;
   }
-  if (tid == 0) {
+  if (warp == 0) {
     const uint64_t dA = sdesc(aQK, 16, 1024), dB = sdesc(aQK + 8192, 16, 1024);
     const uint32_t id = idesc_bf16(128, 64);
 #pragma unroll
     for (int ks = 0; ks < kDK / 16; ++ks)
-      mma_bf16(tb, kstep(dA, 128, ks), kstep(dB, 128, ks), id, ks > 0);
-    mma_commit(mma_bar);
+      mma_bf16_w(tb, kstep(dA, 128, ks), kstep(dB, 128, ks), id, ks > 0);
+    mma_commit_w(mma_bar);
   }
-  __syncwarp();
   if (!mbar_wait(mma_bar, 0, spin_limit)) {
     mbar_wait(mma_bar, 0, kDrainLimit);
     failed = true;
@@ -645,17 +644,17 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       fence_before_sync();
       named_bar(1, 128);
-      if (tid == 0) {
+      if (warp == 0) {
         fence_after_sync();
         const uint64_t dQK = sdesc(a + S_QK, 16, 1024);
         const uint32_t id = idesc_bf16(128, 32);
 #pragma unroll
         for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSH, kDVS, ks), id, ks > 0);
+          mma_bf16_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSH, kDVS, ks), id, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSL, kDVS, ks), id, true);
-        mma_commit(mma_bar);
+          mma_bf16_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSL, kDVS, ks), id, true);
+        mma_commit_w(mma_bar);
       }
       if ((aborted = wait_mma())) break;
       // ---- R = V - Diag(e^G) Y as the operand [v][j] (Y rows: TMEM lanes 64-127) ----------
@@ -685,14 +684,14 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       fence_before_sync();
       named_bar(1, 128);
       // ---- U = T R (tf32) ----------------------------------------------------------------------
-      if (tid == 0) {
+      if (warp == 0) {
         fence_after_sync();
         const uint64_t dT = sdesc(a + S_PT + WS_T, 16, 1024);
         const uint32_t id = idesc_tf32(64, 32, false, false);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
-        mma_commit(mma_bar);
+          mma_tf32_w(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
+        mma_commit_w(mma_bar);
       }
       if ((aborted = wait_mma())) break;
       // ---- U (tf32 [v][j]) and U' = Diag(e^{G_last-G}) U (bf16 hi+lo [v][j]) ------------------
@@ -718,28 +717,30 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       fence_before_sync();
       named_bar(1, 128);
       // ---- O2 = P U (tf32);  S^T += K^T (U'_hi + U'_lo) (bf16) ----------------------------------
-      if (tid == 0) {
+      if (warp == 0) {
+        // the state update first: the chain continues as soon as it completes, while
+        // P U (needed only for the outputs) runs behind it; the stage is released and
+        // the outputs handed to the loader when both have completed
         fence_after_sync();
         const uint64_t dP = sdesc(a + S_PT, 16, 1024);
         const uint64_t dKT = sdesc(a + S_KT, 16, 1024);
-        const uint32_t it = idesc_tf32(64, 32, false, false);
-#pragma unroll
-        for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), it, ks > 0);
         const uint32_t ib = idesc_bf16(128, 32);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
-          mma_bf16(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPH, kDVS, ks), ib, true);
+          mma_bf16_w(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPH, kDVS, ks), ib, true);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
-          mma_bf16(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPL, kDVS, ks), ib, true);
-        mma_commit(mma_bar);
+          mma_bf16_w(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPL, kDVS, ks), ib, true);
+        mma_commit_w(mma_bar);
+        const uint32_t it = idesc_tf32(64, 32, false, false);
+#pragma unroll
+        for (int ks = 0; ks < kC / 8; ++ks)
+          mma_tf32_w(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), it, ks > 0);
+        mma_commit_w(reinterpret_cast<uint64_t*>(&cs.empty[s]));
+        mma_commit_w(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
       }
       if ((aborted = wait_mma())) break;
-      if (tid == 0) {
-        mbar_arrive(reinterpret_cast<uint64_t*>(&cs.empty[s]));
-        mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
-      }      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
+      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
       tmem_ld32(tb + tlane + TM_S, st);
       tmem_wait_ld();
       write_state_operand();
