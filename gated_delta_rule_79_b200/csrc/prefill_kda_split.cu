@@ -219,20 +219,54 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) ps.wmask[q4] = wm;
   }
   tmem_st32(tb + tlane + P_TM_GS + 32 * hw, g);
-  // ---- 3. Gram factors ----------------------------------------------------------------
+  // ---- 3. Gram factors L, R (shared memory) and the carry's images (workspace) ----------
+  // Element (row r, channel cc) of a 128-byte-swizzled K-major tile sits at
+  //   (cc / 32) * rows * 128 + r * 128 + (((cc % 32) / 4 ^ r % 8) * 16) + (cc % 4) * 4;
+  // for this thread's rows r = 32 hw + x only x varies, so the offsets are a per-thread
+  // base for each x % 8 plus 128 x.
+  {
+    const uint32_t ch = (uint32_t)(cc & 31) >> 2;
+    uint32_t o8[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+    for (int kx = 0; kx < 8; ++kx)
+      o8[kx] = (uint32_t)(cc >> 5) * 16384u + (uint32_t)(cc & 3) * 4u + 4096u * hw +
+               ((ch ^ (uint32_t)kx) << 4);
+    unsigned char* rs = tR - (cc >> 5) * 8192;      // R has 64 rows: panel stride 8 KB
+    unsigned char* iqk = img + WS_QK;
+    unsigned char* ikh = img + WS_KH;
+    const float egl = __expf(glast - gm);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int x = 2 * i + u, t = 32 * hw + x;
-      const float qv = u ? bf16_hi(qp[i]) : bf16_lo(qp[i]);
-      const float kv = u ? bf16_hi(kp[i]) : bf16_lo(kp[i]);
-      const float e = wc ? 0.f : __expf(g[x] - gm);
-      const float ei = wc ? 0.f : __expf(gm - g[x]);
-      st_tile(tL, 128, t, cc, qv * e);
-      st_tile(tL, 128, 64 + t, cc, kv * e);
-      st_tile(tR, 64, t, cc, kv * ei);
+    for (int x4 = 0; x4 < 8; ++x4) {
+      float kh[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int x = 4 * x4 + u, t = 32 * hw + x;
+        const uint32_t p2 = qp[x >> 1], k2 = kp[x >> 1];
+        const float qv = (x & 1) ? bf16_hi(p2) : bf16_lo(p2);
+        const float kv = (x & 1) ? bf16_hi(k2) : bf16_lo(k2);
+        const uint32_t off = o8[x & 7] + 128u * (uint32_t)x;
+        float e, ei, eg, el;
+        if (!wc) {
+          e = __expf(g[x] - gm);
+          ei = __expf(gm - g[x]);
+          el = egl * ei;                     // e^{G_last - G}, at most 1
+        } else {
+          e = 0.f;
+          ei = 0.f;
+          el = __expf(fminf(glast - g[x], 0.f));
+        }
+        eg = __expf(g[x]);
+        *reinterpret_cast<float*>(tL + off) = to_tf32(qv * e);
+        *reinterpret_cast<float*>(tL + off + 8192) = to_tf32(kv * e);
+        *reinterpret_cast<float*>(rs + off) = to_tf32(kv * ei);
+        *reinterpret_cast<float*>(iqk + off) = to_tf32(qv * eg);
+        *reinterpret_cast<float*>(iqk + off + 8192) = to_tf32(kv * eg);
+        kh[u] = t < L ? kv * el : 0.f;
+      }
+      *reinterpret_cast<float4*>(ikh + swz_off4(cc, 8 * hw + x4, 128)) =
+          tf32x4(kh[0], kh[1], kh[2], kh[3]);
     }
+    if (hw == 0) reinterpret_cast<float*>(img + WS_EGL)[cc] = __expf(glast);
   }
   tmem_wait_st();
   fence_smem_to_async();
@@ -240,6 +274,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   fence_after_sync();
   const bool anywide = (ps.wmask[0] | ps.wmask[1] | ps.wmask[2] | ps.wmask[3]) != 0u;
+  // ---- 4. the decayed Gram on the tensor cores ------------------------------------------
   if (warp == 0) {
     const uint64_t dL = sdesc(smem_u32(tL), 16, 1024), dR = sdesc(smem_u32(tR), 16, 1024);
     const uint32_t id = idesc_tf32(128, 64, false, false);
@@ -247,30 +282,6 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int ks = 0; ks < kDK / 8; ++ks)
       mma_tf32_w(tb + P_TM_G, kstep(dL, 128, ks), kstep(dR, 64, ks), id, ks > 0);
     mma_commit_w(mma_bar);
-  }
-  // ---- 4. while the Gram runs: the carry's [Q~; K~], e^{G_last} and K^ images -------------
-  {
-    unsigned char* iqk = img + WS_QK;
-    float kh[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int x = 2 * i + u, t = 32 * hw + x;
-        const float qv = u ? bf16_hi(qp[i]) : bf16_lo(qp[i]);
-        const float kv = u ? bf16_hi(kp[i]) : bf16_lo(kp[i]);
-        const float e = __expf(g[x]);
-        *reinterpret_cast<float*>(iqk + swz_off(t, cc, 128)) = to_tf32(qv * e);
-        *reinterpret_cast<float*>(iqk + swz_off(64 + t, cc, 128)) = to_tf32(kv * e);
-        kh[x] = t < L ? kv * __expf(fminf(glast - g[x], 0.f)) : 0.f;
-      }
-    }
-    if (hw == 0) reinterpret_cast<float*>(img + WS_EGL)[cc] = __expf(glast);
-    unsigned char* ikh = img + WS_KH;
-#pragma unroll
-    for (int x = 0; x < 8; ++x)
-      *reinterpret_cast<float4*>(ikh + swz_off4(cc, 8 * hw + x, 128)) =
-          tf32x4(kh[4 * x], kh[4 * x + 1], kh[4 * x + 2], kh[4 * x + 3]);
   }
   bool failed = false;
   if (!mbar_wait(mma_bar, 0, spin_limit)) {
@@ -593,6 +604,8 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
           if (g == 1) tma_load_4d(sbase_u + C_V, &tm_v, v0, h, c * kC, b, full + g);
           issued |= 1 << g;
         }
+        // the next chunk's image heads for L2 now, so that its copies come from there
+        if (c + 1 < nchunks) bulk_prefetch_l2(src + kChunkWs, kChunkWs);
       }
       named_bar(2, 128);
       if (cs.abort) break;
@@ -666,12 +679,13 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
           mma_tf32_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSS, kDVS, ks), id, ks > 0);
         mma_commit_w(mma_bar);
         mma_commit_w(empty + 0);
-        if (lane == 0 && !mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
-        __syncwarp();
       }
       if ((aborted = wait_mma())) break;
       // ---- R = V - Y as the operand [v][j] (Y rows: TMEM lanes 64-127) ------------------------
-      if (q4 >= 2) {
+      // group C (T and v) is waited for by the threads that read v, and by warp 0 before
+      // it issues T R
+      if (q4 >= 2 && !mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
+      if (q4 >= 2 && !cs.abort) {
         const int j = 32 * (q4 - 2) + lane;
         float y[32], vv[32];
         const uint4* vrow = reinterpret_cast<const uint4*>(sm + C_V + j * 64);
@@ -696,6 +710,8 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       named_bar(1, 128);
       // ---- U = T R ---------------------------------------------------------------------------
       if (warp == 0) {
+        if (lane == 0 && !mbar_wait(full + 1, par, spin_limit)) give_up(full + 1, par, true);
+        __syncwarp();
         fence_after_sync();
         const uint32_t id = idesc_tf32(64, 32, false, false);
 #pragma unroll
@@ -703,8 +719,6 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
           mma_tf32_w(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
         mma_commit_w(mma_bar);
         mma_commit_w(empty + 1);
-        if (lane == 0 && !mbar_wait(full + 2, par, spin_limit)) give_up(full + 2, par, true);
-        __syncwarp();
       }
       if ((aborted = wait_mma())) break;
       {
@@ -724,6 +738,8 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       if (warp == 0) {
         // the state update first: the chain continues as soon as it completes, while
         // P U (needed only for the outputs) runs behind it
+        if (lane == 0 && !mbar_wait(full + 2, par, spin_limit)) give_up(full + 2, par, true);
+        __syncwarp();
         fence_after_sync();
         const uint32_t i64 = idesc_tf32(64, 32, false, false);
         const uint32_t i128 = idesc_tf32(128, 32, false, false);
