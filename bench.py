@@ -54,6 +54,12 @@ def algorithmic(w):
     state = w.B * w.H * w.dv * w.dk * 4
     if w.decode:
         return 2 * state * w.T, th * 6 * w.dk * w.dv
+    if w.verify:
+        # state read once, one full snapshot written per token, plus the token inputs
+        # and outputs (small next to the state)
+        a_bytes = 4 * (w.dk if w.mixer == "kda" else 1)
+        per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
+        return (1 + w.T) * state + th * per_th, th * 6 * w.dk * w.dv
     a_bytes = 4 * (w.dk if w.mixer == "kda" else 1)
     per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
     nbytes = th * per_th + state + (state if w.state == "randn" else 0)
@@ -258,6 +264,30 @@ class DecodeRunner:
                     o=self.o)
 
 
+class VerifyRunner:
+    """One multi-token verify call per step (K tokens for every sequence and head,
+    all K snapshots written); the 0.5 GB state and the snapshots exceed L2."""
+
+    def __init__(self, w, dev, seed):
+        import gated_delta_rule_79_b200 as g
+        self.g, self.w, self.dev = g, w, dev
+        self.fn = g.kda_verify if w.mixer == "kda" else g.gdn_verify
+        self.x = device_inputs(w, dev, seed=seed)
+        self.snaps = torch.empty((w.T, w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+        self.o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 1
+        self.kernels = ["verify_kernel"]
+        self.kernel_key = f"verify:{w.name}"
+        self.path = "verify (CUDA cores, fp32 state, K snapshots)"
+        self.l2_note = (f"state of {self.x['s0'].numel() * 4 / 2**20:.0f} MiB and "
+                        f"{self.snaps.numel() * 4 / 2**20:.0f} MiB of snapshots > L2")
+
+    def step(self, i):
+        x = self.x
+        self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], snapshots=self.snaps,
+                o=self.o)
+
+
 def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
     """Warm up, then time exactly `steps` steps with CUDA events on the launching
     stream, bracketed by a barrier and a synchronize on both sides.  Also records
@@ -282,7 +312,7 @@ def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
           for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    per_kernel = not runner.w.decode
+    per_kernel = not (runner.w.decode or runner.w.verify)
     if per_kernel:
         runner.g.timing_start()
     t0.record(stream)
@@ -321,6 +351,23 @@ def time_e2e(w, dev, steps, warmup, seed):
                     dbuf[key].copy_(host[key][t], non_blocking=True)
                 fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o)
                 o_host[t].copy_(o, non_blocking=True)
+    elif w.verify:
+        fn = g.kda_verify if w.mixer == "kda" else g.gdn_verify
+        keys = ("q", "k", "v", "alpha", "beta")
+        dbuf = {k: torch.empty_like(x[k]) for k in keys}
+        state = x["s0"]
+        snaps = torch.empty((w.T, w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+        o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = o.numel() * 2
+
+        def step():
+            for key in keys:
+                dbuf[key].copy_(host[key], non_blocking=True)
+            fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state,
+               snapshots=snaps, o=o)
+            o_host.copy_(o, non_blocking=True)
     else:
         fn = g.kda_prefill if w.mixer == "kda" else g.gdn_prefill
         dbuf = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
@@ -361,8 +408,17 @@ def _oracle_slice(args):
     """Run the oracle over one (batch, head) chain for the first `t_sample` tokens."""
     name, b, h, t_sample = args
     import numpy as np  # noqa: F401
-    from oracle import gated_delta_rule, decode_step
+    from oracle import gated_delta_rule, decode_step, verify_steps
     w = WORKLOADS[name]
+    if w.verify:
+        # K tokens per chain are too few to time: run t_sample chains of the K tokens
+        t = time.perf_counter()
+        for i in range(t_sample):
+            x = slice_inputs(w, (b + i) % w.B, h)
+            verify_steps(*[x[k][None, :, None].double().numpy()
+                           for k in ("q", "k", "v", "alpha", "beta")],
+                         x["s0"][None, None].double().numpy())
+        return time.perf_counter() - t
     x = slice_inputs(w.with_(T=t_sample), b, h)
     col = lambda key: x[key][None, :, None].double().numpy()  # noqa: E731
     s0 = None if x["s0"] is None else x["s0"][None, None].double().numpy()
@@ -387,21 +443,29 @@ class OracleTimer:
         import multiprocessing as mp
         self.w = w
         self.cores = min(len(os.sched_getaffinity(0)), w.B * w.H)
-        t_cal = min(w.T, 64)
-        per_token_head = _oracle_slice((w.name, 0, 0, t_cal)) / t_cal
-        self.t_sample = max(1, min(w.T, int(budget_s / max(per_token_head, 1e-9))))
+        if w.verify:
+            # t_sample counts chains of K tokens per process
+            per_chain = _oracle_slice((w.name, 0, 0, 4)) / 4
+            self.t_sample = max(1, int(budget_s / max(per_chain, 1e-9)))
+            self.tokens_per_unit = w.T
+            what = f"{self.t_sample} chains of {w.T} tokens"
+        else:
+            t_cal = min(w.T, 64)
+            per_token_head = _oracle_slice((w.name, 0, 0, t_cal)) / t_cal
+            self.t_sample = max(1, min(w.T, int(budget_s / max(per_token_head, 1e-9))))
+            self.tokens_per_unit = 1
+            what = f"{self.t_sample} tokens"
         self.chains = [(w.name, i // w.H, i % w.H, self.t_sample) for i in range(self.cores)]
         self.pool = mp.get_context("spawn").Pool(processes=self.cores)
         self.pool.map(_oracle_slice, [(w.name, 0, 0, 1)] * self.cores)   # start the workers
-        self.sample = (f"{self.cores} (sequence, head) chains x {self.t_sample} tokens of "
-                       f"{w.name} per pass, fp64 numpy oracle, one spawn process per chain; "
-                       f"tokens/s = token-heads/s / H")
+        self.sample = (f"{self.cores} processes x {what} of {w.name} per pass, fp64 numpy "
+                       f"oracle, one spawn process per core; tokens/s = token-heads/s / H")
 
     def rate(self):
         t0 = time.perf_counter()
         self.pool.map(_oracle_slice, self.chains)
         wall = time.perf_counter() - t0
-        return self.cores * self.t_sample / wall / self.w.H
+        return self.cores * self.t_sample * self.tokens_per_unit / wall / self.w.H
 
     def close(self):
         self.pool.close()
@@ -423,7 +487,7 @@ def main():
     w = WORKLOADS[a.workload]
     if w.name == "gdn_seq_f32":
         raise SystemExit("gdn_seq_f32 is a parity case, not a bench line")
-    default_steps = 5 if (w.decode or w.name == "kda_long") else 50
+    default_steps = 5 if (w.decode or w.name == "kda_long") else 20 if w.verify else 50
     steps = a.steps if a.steps is not None else default_steps
     warmup = max(3, a.warmup if a.warmup is not None else 5)
     rank, world, local = dist_env()
@@ -457,7 +521,8 @@ def main():
     torch.cuda.set_device(dev)
     active = dist_init(world, "nccl")
     peaks, peak_kind = load_peaks()
-    runner = (DecodeRunner if w.decode else PrefillRunner)(w, dev, seed=1000 * rank)
+    runner = (DecodeRunner if w.decode else VerifyRunner if w.verify
+              else PrefillRunner)(w, dev, seed=1000 * rank)
     clocks = ClockSampler(dev.index)
     clocks.start()
     total_ms, per, kernel_ms = time_device(runner, steps, warmup, dev, active)
@@ -493,7 +558,7 @@ def main():
         dom = max(range(len(kernel_ms)), key=lambda i: kernel_ms[i])
         roofline["dominant"] = runner.kernels[dom] if dom < len(runner.kernels) else None
     extra = {}
-    if not w.decode:
+    if not (w.decode or w.verify):
         extra["roofline_tensor"] = {
             "bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],

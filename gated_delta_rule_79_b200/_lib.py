@@ -22,7 +22,8 @@ CHUNK = 64
 
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
-           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop"]
+           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop",
+           "gdn_verify", "kda_verify"]
 
 
 class GdrError(RuntimeError):
@@ -52,6 +53,10 @@ def _load():
         f = getattr(lib, name)
         f.restype = i
         f.argtypes = [vp, vp, vp, fp, fp, fp, vp, i, i, i, i, i, i, vp]
+    for name in ("gdn_verify", "kda_verify"):
+        f = getattr(lib, name)
+        f.restype = i
+        f.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, i, vp]
     lib.gdn_prefill_noalloc.restype = i
     lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdr_prefill_path.restype = i
@@ -214,6 +219,57 @@ def gdn_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=No
 def kda_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
     """One Kimi Delta Attention decode step (alpha [N, H, d_k]); as ``gdn_decode``."""
     return _decode(True, q, k, v, alpha, beta, state, out_dtype, o, stream)
+
+
+VERIFY_MAX_TOKENS = 16
+
+
+def _verify(kda, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream):
+    if q.dim() != 4:
+        raise ValueError("q must be [N, K, H, d_k]")
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    dt = q.dtype
+    _need(q, "q", (N, K, H, dk), dt, dev)
+    _need(k, "k", (N, K, H, dk), dt, dev)
+    _need(v, "v", (N, K, H, dv), dt, dev)
+    _need(alpha, "alpha", (N, K, H, dk) if kda else (N, K, H), torch.float32, dev)
+    _need(beta, "beta", (N, K, H), torch.float32, dev)
+    _need(state, "state", (N, H, dv, dk), torch.float32, dev)
+    if snapshots is True:
+        snapshots = torch.empty((K, N, H, dv, dk), dtype=torch.float32, device=dev)
+    elif snapshots is False:
+        snapshots = None
+    if snapshots is not None:
+        _need(snapshots, "snapshots", (K, N, H, dv, dk), torch.float32, dev)
+    out_dtype = out_dtype or dt
+    if o is None:
+        o = torch.empty((N, K, H, dv), dtype=out_dtype, device=dev)
+    _need(o, "o", (N, K, H, dv), out_dtype, dev)
+    fn = lib.kda_verify if kda else lib.gdn_verify
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(snapshots),
+              _ptr(o), N, K, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream)))
+    return o, snapshots
+
+
+def gdn_verify(q, k, v, alpha, beta, state, *, snapshots=True, out_dtype=None, o=None,
+               stream=None):
+    """Gated DeltaNet over K tokens per sequence from a carried state, keeping the
+    state after every token.  q, k [N, K, H, d_k]; v [N, K, H, d_v]; alpha, beta
+    [N, K, H]; state [N, H, d_v, d_k] float32.  snapshots=True allocates, or pass a
+    [K, N, H, d_v, d_k] float32 tensor; snapshots[t] is the state after token t+1 and
+    ``state`` is left as it was.  snapshots=False updates ``state`` in place to the
+    state after the K tokens instead.  Returns (o [N, K, H, d_v], snapshots or None)."""
+    return _verify(False, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream)
+
+
+def kda_verify(q, k, v, alpha, beta, state, *, snapshots=True, out_dtype=None, o=None,
+               stream=None):
+    """Kimi Delta Attention (alpha [N, K, H, d_k]); as ``gdn_verify``."""
+    return _verify(True, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream)
 
 
 def prefill_path(dk, dv, dtype, kda):

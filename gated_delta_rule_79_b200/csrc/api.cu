@@ -121,6 +121,38 @@ static gdr_status decode(bool kda, const void* q, const void* k, const void* v,
   return ok();
 }
 
+static gdr_status verify(bool kda, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* beta, float* state, float* snapshots,
+                         void* o, int N, int K, int H, int dk, int dv, int in_dtype,
+                         int out_dtype, void* stream) {
+  const char* fn = kda ? "kda_verify" : "gdn_verify";
+  if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "%s: negative size N=%d H=%d", fn, N, H);
+  if (K < 1 || K > GDR_VERIFY_MAX_TOKENS)
+    return fail(GDR_ERR_UNSUPPORTED, "%s: K=%d tokens (supported: 1 to %d)", fn, K,
+                GDR_VERIFY_MAX_TOKENS);
+  if (!head_ok(dk) || !head_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "%s: d_k=%d d_v=%d (supported: 32, 64, 128)", fn, dk, dv);
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype))
+    return fail(GDR_ERR_INVALID_ARG, "%s: bad dtype in=%d out=%d", fn, in_dtype, out_dtype);
+  if ((long long)N * H > (1LL << 31) / 4 || (long long)N * H * K * (dk > dv ? dk : dv) > (1LL << 40))
+    return fail(GDR_ERR_INVALID_ARG, "%s: N*H too large", fn);
+  if (N == 0 || H == 0) return ok();
+  const void* need_ptrs[] = {q, k, v, alpha, beta, state, o};
+  const char* names[] = {"q", "k", "v", "alpha", "beta", "state", "o"};
+  for (int i = 0; i < 7; ++i) {
+    if (!need_ptrs[i]) return fail(GDR_ERR_INVALID_ARG, "%s: %s is NULL", fn, names[i]);
+    if (!aligned16(need_ptrs[i]))
+      return fail(GDR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
+  }
+  if (snapshots && !aligned16(snapshots))
+    return fail(GDR_ERR_INVALID_ARG, "%s: snapshots is not 16-byte aligned", fn);
+  VerifyArgs a{q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv,
+               in_dtype, out_dtype, kda};
+  cudaError_t e = launch_verify(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return ok();
+}
+
 }  // namespace gdr
 
 extern "C" {
@@ -163,6 +195,20 @@ gdr_status kda_decode(const void* q, const void* k, const void* v, const float* 
                       int in_dtype, int out_dtype, void* stream) {
   return gdr::decode(true, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
                      stream);
+}
+
+gdr_status gdn_verify(const void* q, const void* k, const void* v, const float* alpha,
+                      const float* beta, float* state, float* snapshots, void* o, int N, int K,
+                      int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
+  return gdr::verify(false, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
+                     out_dtype, stream);
+}
+
+gdr_status kda_verify(const void* q, const void* k, const void* v, const float* alpha,
+                      const float* beta, float* state, float* snapshots, void* o, int N, int K,
+                      int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
+  return gdr::verify(true, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
+                     out_dtype, stream);
 }
 
 int gdr_prefill_path(int dk, int dv, int in_dtype, int kda) {

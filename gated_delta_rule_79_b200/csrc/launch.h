@@ -36,6 +36,20 @@ struct DecodeArgs {
   bool kda;
 };
 
+struct VerifyArgs {
+  const void* q;        // [N, K, H, dk]
+  const void* k;
+  const void* v;        // [N, K, H, dv]
+  const float* alpha;   // [N, K, H] or [N, K, H, dk]
+  const float* beta;    // [N, K, H]
+  float* state;         // [N, H, dv, dk]: read; updated in place when snapshots is null
+  float* snapshots;     // [K, N, H, dv, dk] or null
+  void* o;              // [N, K, H, dv]
+  int N, K, H, dk, dv;
+  int in_dtype, out_dtype;
+  bool kda;
+};
+
 // Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
 int report_error(int s, const char* msg);
 
@@ -45,6 +59,7 @@ void timing_mark(cudaStream_t stream, int slot);
 
 // Each returns cudaSuccess or the launch error; messages are set by the caller.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
 
 }  // namespace gdr

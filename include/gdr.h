@@ -160,6 +160,42 @@ GDR_API gdr_status gdn_prefill_noalloc(const void* q, const void* k, const void*
                        int B, int T, int H, int dk, int dv,
                        int in_dtype, int out_dtype, int chunk, void* stream);
 
+/* Largest number of tokens per (sequence, head) that gdn_verify / kda_verify take. */
+#define GDR_VERIFY_MAX_TOKENS 16
+
+/* Multi-token step from a carried state, keeping the state after every token.
+ * "Super Apriel: One Checkpoint, Many Speeds", §2D (inference and serving) and §4
+ * (speculative decoding): the all-GDN placement drafts tokens that the all-FA placement
+ * verifies, with no separate draft model, so a recurrent mixer must be able to run K
+ * tokens from its state and then continue from whichever of them was the last one
+ * accepted.  For each of N sequences and H heads this runs the recurrence over K tokens
+ * (1 <= K <= GDR_VERIFY_MAX_TOKENS) starting from `state`:
+ *
+ *   q, k       [N, K, H, d_k]   in_dtype
+ *   v          [N, K, H, d_v]   in_dtype
+ *   alpha      GDN: [N, K, H] fp32;  KDA: [N, K, H, d_k] fp32
+ *   beta       [N, K, H] fp32
+ *   state      [N, H, d_v, d_k] fp32, the state before the first token
+ *   snapshots  [K, N, H, d_v, d_k] fp32 (written): snapshots[t] is the whole state
+ *              after token t+1, so the caller adopts snapshots[m-1] after accepting m
+ *              tokens without a copy; `state` is then only read.  NULL: no snapshots,
+ *              and `state` is updated in place to the state after the K tokens (a
+ *              K-token decode).  Must not overlap state or the inputs.
+ *   o          [N, K, H, d_v]   out_dtype (written), o[n, t] = S_{t+1} q_t
+ *
+ * N or H equal to 0 is a valid empty call.  No workspace is used.  Same head sizes and
+ * dtypes as the decode entry points. */
+GDR_API gdr_status gdn_verify(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, float* snapshots,
+                      void* o, int N, int K, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream);
+
+/* Same contract as gdn_verify with the per-channel gate alpha [N, K, H, d_k]. */
+GDR_API gdr_status kda_verify(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, float* snapshots,
+                      void* o, int N, int K, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream);
+
 /* Which prefill kernel a call with these parameters runs: 1 = the bf16
  * tensor-core (tcgen05) kernel, 0 = the fp32 CUDA-core kernel, -1 = the
  * parameters are not supported.  Pure host query, no CUDA call. */

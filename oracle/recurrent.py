@@ -88,3 +88,29 @@ def decode_step(q, k, v, alpha, beta, state):
                             _as_f64(v)[:, None], _as_f64(alpha)[:, None],
                             _as_f64(beta)[:, None], state)
     return o[:, 0], s
+
+
+def verify_steps(q, k, v, alpha, beta, state):
+    """K tokens per sequence from a carried state, keeping the state after each token.
+
+    "Super Apriel: One Checkpoint, Many Speeds", §2D and §4 (speculative decoding):
+    the all-GDN placement drafts tokens for the all-FA placement to verify, so a
+    recurrent mixer must be able to resume from any of K tokens.  By definition the
+    snapshot after token t is the state the recurrence reaches after the first t
+    tokens, and the outputs are those of the same run.
+
+      q, k [N, K, H, d_k]; v [N, K, H, d_v]; alpha [N, K, H] or [N, K, H, d_k];
+      beta [N, K, H]; state [N, H, d_v, d_k] (not modified).
+    Returns (o [N, K, H, d_v], snapshots [K, N, H, d_v, d_k]) in fp64.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    alpha, beta = _as_f64(alpha), _as_f64(beta)
+    K = q.shape[1]
+    S = _as_f64(state)
+    outs, snaps = [], []
+    for t in range(K):
+        o, S = gated_delta_rule(q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1],
+                                alpha[:, t:t + 1], beta[:, t:t + 1], S)
+        outs.append(o[:, 0])
+        snaps.append(S)
+    return np.stack(outs, axis=1), np.stack(snaps, axis=0)

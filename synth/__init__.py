@@ -12,6 +12,8 @@ Workloads (all inputs synthetic; the pages publish no dataset for the mixer):
   decode        N=256 sequences x H=32, d=128, 512 one-token steps, bf16
                 q/k/v, fp32 state ~ 0.02 N(0,1); GDN and KDA gates
   kda_long      KDA, B=4 H=32 T=65536 d=128, bf16, state ~ 0.02 N(0,1)
+  verify_gdn    N=256 sequences x H=32, d=128, K=4 tokens from a carried state
+  verify_kda    ~ 0.02 N(0,1), bf16 q/k/v; GDN and KDA gates (B = N, T = K)
 
 Recipe per (batch b, head h) slice, one ``torch.Generator`` (CPU) seeded with
 ``slice_seed(seed, b, h)``, drawing in this fixed order:
@@ -50,6 +52,7 @@ class Workload:
     dtype: str          # "f32" or "bf16" for q, k, v
     state: str          # "zeros" or "randn"
     decode: bool = False
+    verify: bool = False  # K tokens (the T axis) from a carried state, snapshots kept
 
     @property
     def torch_dtype(self):
@@ -66,6 +69,10 @@ WORKLOADS = {
     "decode_gdn": Workload("decode_gdn", "gdn", 256, 32, 512, 128, 128, "bf16", "randn", True),
     "decode_kda": Workload("decode_kda", "kda", 256, 32, 512, 128, 128, "bf16", "randn", True),
     "kda_long": Workload("kda_long", "kda", 4, 32, 65536, 128, 128, "bf16", "randn"),
+    "verify_gdn": Workload("verify_gdn", "gdn", 256, 32, 4, 128, 128, "bf16", "randn",
+                           verify=True),
+    "verify_kda": Workload("verify_kda", "kda", 256, 32, 4, 128, 128, "bf16", "randn",
+                           verify=True),
 }
 
 

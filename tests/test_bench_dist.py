@@ -69,3 +69,14 @@ def test_two_rank_gloo_max_and_aggregate():
         assert active
         assert mx == 150.0                          # max over ranks, not the local time
         assert value == pytest.approx(4096 * 2 / 0.150)
+
+
+def test_verify_algorithmic_bytes_count_state_and_snapshots():
+    """A verify call reads the state once and writes one full snapshot per token."""
+    import bench
+    from synth import WORKLOADS
+    w = WORKLOADS["verify_gdn"]
+    state = w.B * w.H * w.dv * w.dk * 4
+    nb, flops = bench.algorithmic(w)
+    assert (1 + w.T) * state < nb < (1 + w.T) * state * 1.02
+    assert flops == w.B * w.T * w.H * 6 * w.dk * w.dv

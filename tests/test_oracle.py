@@ -346,3 +346,69 @@ def test_decode_does_not_modify_input_state():
     keep = S0.copy()
     decode_step(q[:, 0], k[:, 0], v[:, 0], alpha[:, 0], beta[:, 0], S0)
     assert np.array_equal(S0, keep)
+
+
+# --------------------------------------------------------------------------------------
+# verify_steps: K tokens from a carried state with the state after each token
+
+from oracle import verify_steps  # noqa: E402
+
+
+def _verify_case(kda, N=2, K=5, H=3, dk=4, dv=3, seed=31, **kw):
+    q, k, v, alpha, beta, S0 = _rand_case(B=N, T=K, H=H, dk=dk, dv=dv, kda=kda,
+                                          rng=np.random.default_rng(seed), **kw)
+    return q, k, v, alpha, beta, S0
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_verify_snapshots_match_the_chunked_restatement(kda):
+    """Snapshot t is the state after the first t+1 tokens, and the outputs are those
+    of the same run: checked against the independent chunk-wise code."""
+    q, k, v, alpha, beta, S0 = _verify_case(kda)
+    o, snaps = verify_steps(q, k, v, alpha, beta, S0)
+    assert o.shape == (2, 5, 3, 3) and snaps.shape == (5, 2, 3, 3, 4)
+    for t in range(q.shape[1]):
+        oc, sc = chunked_gated_delta_rule(q[:, :t + 1], k[:, :t + 1], v[:, :t + 1],
+                                          alpha[:, :t + 1], beta[:, :t + 1], S0, chunk=4)
+        assert np.allclose(snaps[t], sc, rtol=1e-12, atol=1e-12)
+        assert np.allclose(o[:, :t + 1], oc, rtol=1e-12, atol=1e-12)
+
+
+def test_verify_identity_gates_keep_the_state():
+    """alpha = 1, beta = 0: every snapshot is S0 and o_t = S0 q_t exactly."""
+    q, k, v, alpha, beta, S0 = _verify_case(True)
+    alpha = np.ones_like(alpha)
+    beta = np.zeros_like(beta)
+    o, snaps = verify_steps(q, k, v, alpha, beta, S0)
+    for t in range(q.shape[1]):
+        assert np.array_equal(snaps[t], S0)
+        assert np.allclose(o[:, t], np.einsum("nhvk,nhk->nhv", S0, q[:, t]), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_verify_read_back_after_every_token(kda):
+    """beta = 1 and unit k: the state after token t maps k_t to v_t, whatever the gates."""
+    q, k, v, alpha, beta, S0 = _verify_case(kda, seed=32)
+    beta = np.ones_like(beta)
+    _, snaps = verify_steps(q, k, v, alpha, beta, S0)
+    for t in range(q.shape[1]):
+        assert np.allclose(np.einsum("nhvk,nhk->nhv", snaps[t], k[:, t]), v[:, t], atol=1e-12)
+
+
+def test_verify_pins_catch_an_off_by_one_snapshot():
+    """A planted mistake (recording the state before each token instead of after it)
+    fails the read-back pin."""
+    q, k, v, alpha, beta, S0 = _verify_case(False, seed=33)
+    beta = np.ones_like(beta)
+    _, snaps = verify_steps(q, k, v, alpha, beta, S0)
+    wrong = np.concatenate([S0[None], snaps[:-1]], axis=0)
+    ok = all(np.allclose(np.einsum("nhvk,nhk->nhv", wrong[t], k[:, t]), v[:, t], atol=1e-12)
+             for t in range(q.shape[1]))
+    assert not ok
+
+
+def test_verify_leaves_the_input_state():
+    q, k, v, alpha, beta, S0 = _verify_case(True, seed=34)
+    keep = S0.copy()
+    verify_steps(q, k, v, alpha, beta, S0)
+    assert np.array_equal(S0, keep)
