@@ -23,7 +23,8 @@ CHUNK = 64
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
            "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop",
-           "gdn_verify", "kda_verify"]
+           "gdn_verify", "kda_verify", "gdr_prefill_varlen_workspace_bytes",
+           "gdn_prefill_varlen", "kda_prefill_varlen"]
 
 
 class GdrError(RuntimeError):
@@ -57,6 +58,12 @@ def _load():
         f = getattr(lib, name)
         f.restype = i
         f.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, i, i, i, i, i, i, i, vp]
+    lib.gdr_prefill_varlen_workspace_bytes.restype = sz
+    lib.gdr_prefill_varlen_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    for name in ("gdn_prefill_varlen", "kda_prefill_varlen"):
+        f = getattr(lib, name)
+        f.restype = i
+        f.argtypes = [vp, vp, vp, fp, fp, vp, vp, fp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
     lib.gdn_prefill_noalloc.restype = i
     lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdr_prefill_path.restype = i
@@ -219,6 +226,68 @@ def gdn_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=No
 def kda_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
     """One Kimi Delta Attention decode step (alpha [N, H, d_k]); as ``gdn_decode``."""
     return _decode(True, q, k, v, alpha, beta, state, out_dtype, o, stream)
+
+
+def _prefill_varlen(kda, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
+                    chunk, stream, workspace):
+    if q.dim() != 3:
+        raise ValueError("q must be [total, H, d_k] (sequences packed along the tokens)")
+    total, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    dt = q.dtype
+    _need(q, "q", (total, H, dk), dt, dev)
+    _need(k, "k", (total, H, dk), dt, dev)
+    _need(v, "v", (total, H, dv), dt, dev)
+    _need(alpha, "alpha", (total, H, dk) if kda else (total, H), torch.float32, dev)
+    _need(beta, "beta", (total, H), torch.float32, dev)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != dev:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor on the inputs' device")
+    nseq = cu_seqlens.numel() - 1
+    if nseq < 0:
+        raise ValueError("cu_seqlens needs nseq + 1 entries")
+    if state.dim() != 4 or state.shape[1:] != (H, dv, dk) or state.dtype != torch.float32:
+        raise ValueError("state must be a float32 pool [nslots, H, d_v, d_k]")
+    if not state.is_contiguous() or state.device != dev:
+        raise ValueError("state must be contiguous on the inputs' device")
+    if slots is not None and (slots.dtype != torch.int32 or slots.numel() != nseq
+                              or slots.device != dev):
+        raise ValueError("slots must be an int32 tensor of nseq entries on the inputs' device")
+    if slots is None and state.shape[0] < nseq:
+        raise ValueError("without slots the pool needs one slot per sequence")
+    out_dtype = out_dtype or dt
+    if o is None:
+        o = torch.empty((total, H, dv), dtype=out_dtype, device=dev)
+    _need(o, "o", (total, H, dv), out_dtype, dev)
+    need = lib.gdr_prefill_varlen_workspace_bytes(nseq, total, H, dk, dv, int(kda))
+    if workspace is None:
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(s):
+            workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    fn = lib.kda_prefill_varlen if kda else lib.gdn_prefill_varlen
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens), _ptr(slots),
+              _ptr(state), _ptr(o), nseq, total, H, dk, dv, _code(dt), _code(out_dtype), chunk,
+              _ptr(workspace), workspace.numel(), _stream(dev, stream)))
+    return o
+
+
+def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, state, *, slots=None, out_dtype=None,
+                       o=None, chunk=CHUNK, stream=None, workspace=None):
+    """Gated DeltaNet prefill of nseq sequences packed along the tokens: q, k
+    [total, H, d_k], v [total, H, d_v] bf16; alpha, beta [total, H] float32; cu_seqlens
+    int32 [nseq + 1] on the device; state a float32 pool [nslots, H, d_v, d_k] read
+    from and written back to slot slots[i] (default i) in place.  Returns o."""
+    return _prefill_varlen(False, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
+                           chunk, stream, workspace)
+
+
+def kda_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, state, *, slots=None, out_dtype=None,
+                       o=None, chunk=CHUNK, stream=None, workspace=None):
+    """Kimi Delta Attention (alpha [total, H, d_k]); as ``gdn_prefill_varlen``."""
+    return _prefill_varlen(True, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
+                           chunk, stream, workspace)
 
 
 VERIFY_MAX_TOKENS = 16

@@ -232,8 +232,12 @@ gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream) 
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess)
     return gdr::fail(GDR_ERR_CUDA, "gdr_workspace_status: %s", cudaGetErrorString(e));
-  if (word != 0)
+  if (word & 3u)
     return gdr::fail(GDR_ERR_TIMEOUT, "a bounded device wait gave up (status word 0x%08x)", word);
+  if (word != 0)
+    return gdr::fail(GDR_ERR_INVALID_ARG,
+                     "packed-sequence offsets were not a partition of the tokens (status word "
+                     "0x%08x); no chunk was processed", word);
   return gdr::ok();
 }
 

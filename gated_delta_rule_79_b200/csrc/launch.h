@@ -50,6 +50,18 @@ struct VerifyArgs {
   bool kda;
 };
 
+struct ChunkMap;   // chunkmap.cuh
+
+// The two-kernel tensor-core prefills (prefill_split.cu, prefill_kda_split.cu): bf16,
+// d_k = 128, d_v a multiple of 32.  Chunk images per (head, chunk) in the workspace.
+size_t split_prefill_workspace(int B, int T, int H);
+size_t kda_split_workspace(int B, int T, int H);
+size_t split_chunk_image_bytes();
+size_t kda_chunk_image_bytes();
+cudaError_t launch_prefill_split(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream);
+cudaError_t launch_prefill_kda_split(const PrefillArgs& a, const ChunkMap& m,
+                                     cudaStream_t stream);
+
 // Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
 int report_error(int s, const char* msg);
 

@@ -38,6 +38,7 @@
 #include <math.h>
 #include <stdlib.h>
 
+#include "chunkmap.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -121,7 +122,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __nv_bfloat16* __restrict__ q,
                       const __nv_bfloat16* __restrict__ k, const float* __restrict__ beta,
-                      unsigned char* __restrict__ ws, int T, int H, int nchunks,
+                      unsigned char* __restrict__ ws, const ChunkMap m, int H,
                       unsigned int* __restrict__ status, uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -138,13 +139,13 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, hw = warp >> 2;
-  const int c = blockIdx.x % nchunks;
-  const int bh = blockIdx.x / nchunks;
-  const int h = bh % H, b = bh / H;
-  const int t0 = c * kC;
-  const int L = min(kC, T - t0);
-  const long row0 = ((long)b * T + t0) * H + h;    // token t of the chunk: row0 + t * H
-  unsigned char* img = ws + kStatusBytes + ((size_t)bh * nchunks + c) * kChunkWs;
+  const int gc = blockIdx.x % m.nck;
+  const int h = blockIdx.x / m.nck;
+  const ChunkLoc loc = chunk_locate(m, gc);
+  if (!loc.valid) return;            // past the last chunk of the packed sequences
+  const int b = loc.b, t0 = loc.t0, L = loc.L;
+  const long row0 = ((long)b * m.T + t0) * H + h;    // token t of the chunk: row0 + t * H
+  unsigned char* img = ws + m.img_base + ((size_t)h * m.nck + gc) * kChunkWs;
 
   // the chunk's q and k (bf16 [64 t][128 c]) land in the L area and its gates (fp32
   // [64 t][128 c]) in the R area; both are read into registers before L and R are built
@@ -474,8 +475,8 @@ template <typename Tout>
 __global__ void __launch_bounds__(C_THREADS, 1)
 kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
                        const unsigned char* __restrict__ ws, const float* __restrict__ s0,
-                       Tout* __restrict__ o, float* __restrict__ s_final, int T, int H, int dv,
-                       int nchunks, unsigned int* __restrict__ status, uint32_t spin_limit) {
+                       Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m,
+                       int H, int dv, unsigned int* __restrict__ status, uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + padb;
@@ -491,8 +492,10 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
   const int q4 = warp & 3;
   const int nslice = dv / kDVS;
   const int slice = blockIdx.x % nslice;
-  const int bh = blockIdx.x / nslice;
-  const int h = bh % H, b = bh / H;
+  const int sh = blockIdx.x / nslice;
+  const int h = sh % H, seq = sh / H;
+  int first = 0, nchunks = 0;
+  chunk_range(m, seq, first, nchunks);
   const int v0 = slice * kDVS;
 
   if (tid == 0) {
@@ -514,7 +517,7 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
   fence_after_sync();
   const uint32_t tb = cs.tmem;
   const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
-  const unsigned char* wsb = ws + kStatusBytes + (size_t)bh * nchunks * kChunkWs;
+  const unsigned char* wsb = ws + m.img_base + ((size_t)h * m.nck + first) * kChunkWs;
   const uint32_t sbase_u = smem_u32(sm);
 
   auto give_up = [&](uint64_t* bar, uint32_t parity, bool drain) {
@@ -534,8 +537,8 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       named_bar(2, 128);
       if (cs.abort) return false;
       fence_after_sync();
-      const int t0 = cc * kC;
-      const int L = min(kC, T - t0);
+      const ChunkLoc loc = chunk_locate(m, first + cc);
+      const int t0 = loc.t0, L = loc.L, b = loc.b;
       {
         float o2[32];
         tmem_ld32(tb + tlane + TM_O2 + 32 * ob, o2);
@@ -555,7 +558,7 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
         for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
         tmem_wait_ld();
         if (t < L) {
-          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
+          Tout* dst = o + (((long)b * m.T + t0 + t) * H + h) * (long)dv + v0;
           if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
@@ -601,7 +604,10 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
           }
           mbar_expect_tx(full + g, bytes[g] + (g == 1 ? 4096u : 0u));
           bulk_load(dst[g], src + off[g], bytes[g], full + g);
-          if (g == 1) tma_load_4d(sbase_u + C_V, &tm_v, v0, h, c * kC, b, full + g);
+          if (g == 1) {
+            const ChunkLoc loc = chunk_locate(m, first + c);
+            tma_load_4d(sbase_u + C_V, &tm_v, v0, h, loc.t0, loc.b, full + g);
+          }
           issued |= 1 << g;
         }
         // the next chunk's image heads for L2 now, so that its copies come from there
@@ -616,10 +622,10 @@ kda_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
       for (int g = 0; g < 3; ++g)
         if (issued & (1 << g)) mbar_wait(full + g, last_par, kDrainLimit);
     }
-    if (!cs.abort) write_outputs(nchunks - 1);
+    if (!cs.abort && nchunks > 0) write_outputs(nchunks - 1);
   } else {
     // =========================== carry warpgroup ======================================
-    const long sbase = ((long)b * H + h) * (long)dv * kDK;
+    const long sbase = ((long)chunk_state_index(m, seq) * H + h) * (long)dv * kDK;
     float st[kDVS];
 #pragma unroll
     for (int vv = 0; vv < kDVS; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
@@ -780,29 +786,30 @@ uint32_t kda_split_spin_limit() {
 }
 
 template <typename Tout>
-cudaError_t launch_kda_split_t(const PrefillArgs& a, cudaStream_t stream) {
+cudaError_t launch_kda_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
+  // packed sequences: the tensors are [1, total, H, *]
+  const int TB = m.cu ? 1 : a.B;
   CUtensorMap mq, mk, ma, mv;
-  if (!encode_bthd_bf16(&mq, a.q, a.B, a.T, a.H, kDK, kDK, kC, false) ||
-      !encode_bthd_bf16(&mk, a.k, a.B, a.T, a.H, kDK, kDK, kC, false) ||
-      !encode_bthd_f32(&ma, a.alpha, a.B, a.T, a.H, kDK, kDK, kC) ||
-      !encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC, false))
+  if (!encode_bthd_bf16(&mq, a.q, TB, a.T, a.H, kDK, kDK, kC, false) ||
+      !encode_bthd_bf16(&mk, a.k, TB, a.T, a.H, kDK, kDK, kC, false) ||
+      !encode_bthd_f32(&ma, a.alpha, TB, a.T, a.H, kDK, kDK, kC) ||
+      !encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, kDVS, kC, false))
     return cudaErrorInvalidValue;
-  const int nchunks = (a.T + kC - 1) / kC;
   const uint32_t lim = kda_split_spin_limit();
   cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  kda_chunk_prep_kernel<<<a.B * a.H * nchunks, P_THREADS, P_SMEM, stream>>>(
+  kda_chunk_prep_kernel<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
       mq, mk, ma, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.beta,
-      (unsigned char*)a.workspace, a.T, a.H, nchunks, (unsigned int*)a.workspace, lim);
+      (unsigned char*)a.workspace, m, a.H, (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   timing_mark(stream, 0);
   auto carry = kda_chunk_carry_kernel<Tout>;
   e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return e;
-  carry<<<a.B * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
-      mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, a.T, a.H, a.dv, nchunks,
+  carry<<<m.nseq * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
+      mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H, a.dv,
       (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e == cudaSuccess) timing_mark(stream, 1);
@@ -816,9 +823,12 @@ size_t kda_split_workspace(int B, int T, int H) {
   return (size_t)B * H * nchunks * kChunkWs;
 }
 
-cudaError_t launch_prefill_kda_split(const PrefillArgs& a, cudaStream_t stream) {
-  if (a.out_dtype == GDR_F32) return launch_kda_split_t<float>(a, stream);
-  return launch_kda_split_t<__nv_bfloat16>(a, stream);
+size_t kda_chunk_image_bytes() { return kChunkWs; }
+
+cudaError_t launch_prefill_kda_split(const PrefillArgs& a, const ChunkMap& m,
+                                     cudaStream_t stream) {
+  if (a.out_dtype == GDR_F32) return launch_kda_split_t<float>(a, m, stream);
+  return launch_kda_split_t<__nv_bfloat16>(a, m, stream);
 }
 
 }  // namespace gdr

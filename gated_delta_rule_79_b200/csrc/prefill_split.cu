@@ -30,6 +30,7 @@
 #include <math.h>
 #include <stdlib.h>
 
+#include "chunkmap.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -103,8 +104,8 @@ struct PrepSmall {
 __global__ void __launch_bounds__(P_THREADS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ alpha,
-                      const float* __restrict__ beta, unsigned char* __restrict__ ws, int T,
-                      int H, int nchunks, unsigned int* __restrict__ status,
+                      const float* __restrict__ beta, unsigned char* __restrict__ ws,
+                      const ChunkMap m, int H, unsigned int* __restrict__ status,
                       uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -121,11 +122,11 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x % nchunks;
-  const int bh = blockIdx.x / nchunks;
-  const int h = bh % H, b = bh / H;
-  const int t0 = c * kC;
-  const int L = min(kC, T - t0);
+  const int gc = blockIdx.x % m.nck;
+  const int h = blockIdx.x / m.nck;
+  const ChunkLoc loc = chunk_locate(m, gc);
+  if (!loc.valid) return;            // past the last chunk of the packed sequences
+  const int b = loc.b, t0 = loc.t0, L = loc.L;
 
   if (tid == 0) {
     mbar_init(tma_bar, 1);
@@ -150,7 +151,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (tid < kC) {
     float a = 1.f, bt = 0.f;
     if (tid < L) {
-      const long row = ((long)b * T + t0 + tid) * H + h;
+      const long row = ((long)b * m.T + t0 + tid) * H + h;
       a = alpha[row];
       bt = beta[row];
     }
@@ -343,7 +344,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   fence_smem_to_async();
   __syncthreads();
   if (tid == 0) {
-    unsigned char* dst = ws + kStatusBytes + ((size_t)bh * nchunks + c) * kChunkWs;
+    unsigned char* dst = ws + m.img_base + ((size_t)h * m.nck + gc) * kChunkWs;
     bulk_store(dst, smem_u32(tP), kChunkWs);
     bulk_commit();
     bulk_wait_all();
@@ -407,8 +408,8 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const unsigned char* __restrict__ ws, const float* __restrict__ s0,
-                       Tout* __restrict__ o, float* __restrict__ s_final, int T, int H, int dv,
-                       int nchunks, unsigned int* __restrict__ status, uint32_t spin_limit) {
+                       Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m,
+                       int H, int dv, unsigned int* __restrict__ status, uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + padb;
@@ -425,8 +426,10 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int q4 = warp & 3;
   const int nslice = dv / kDVS;
   const int slice = blockIdx.x % nslice;
-  const int bh = blockIdx.x / nslice;
-  const int h = bh % H, b = bh / H;
+  const int sh = blockIdx.x / nslice;
+  const int h = sh % H, seq = sh / H;
+  int first = 0, nchunks = 0;
+  chunk_range(m, seq, first, nchunks);
   const int v0 = slice * kDVS;
 
   if (tid == 0) {
@@ -449,7 +452,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
   fence_after_sync();
   const uint32_t tb = cs.tmem;
   const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
-  const unsigned char* wsb = ws + kStatusBytes + (size_t)bh * nchunks * kChunkWs;
+  const unsigned char* wsb = ws + m.img_base + ((size_t)h * m.nck + first) * kChunkWs;
 
   auto stage = [&](int s) { return sm + s * STAGE_BYTES; };
   // A wait gave up: record the timeout and stop both warpgroups.  For barriers fed by
@@ -474,8 +477,8 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       named_bar(2, 128);
       if (cs.abort) return false;
       fence_after_sync();
-      const int t0 = cc * kC;
-      const int L = min(kC, T - t0);
+      const ChunkLoc loc = chunk_locate(m, first + cc);
+      const int t0 = loc.t0, L = loc.L, b = loc.b;
       {
         float o2[32];
         tmem_ld32(tb + tlane + TM_O2 + 32 * ob, o2);
@@ -496,7 +499,7 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float eg = cs.eg_out[ob][t];
         tmem_wait_ld();
         if (t < L) {
-          Tout* dst = o + (((long)b * T + t0 + t) * H + h) * (long)dv + v0;
+          Tout* dst = o + (((long)b * m.T + t0 + t) * H + h) * (long)dv + v0;
           if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -542,7 +545,8 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (cs.abort) break;
       if (lt == 0 && ok) {
         const uint32_t a = smem_u32(st);
-        const int t0 = c * kC;
+        const ChunkLoc loc = chunk_locate(m, first + c);
+        const int t0 = loc.t0, b = loc.b;
         mbar_expect_tx(full, STAGE_TX);
         tma_load_4d(a + S_QK, &tm_q, 0, h, t0, b, full);
         tma_load_4d(a + S_QK + 16384, &tm_q, 64, h, t0, b, full);
@@ -578,11 +582,11 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lt == 0) mbar_arrive(ready);
       if (c > 0 && !write_outputs(c - 1)) break;
     }
-    if (!cs.abort) write_outputs(nchunks - 1);
+    if (!cs.abort && nchunks > 0) write_outputs(nchunks - 1);
   } else {
     // =========================== carry warpgroup ======================================
     // state: thread c < 128 owns row c of S^T (S[v0 + v][c], v < 32)
-    const long sbase = ((long)b * H + h) * (long)dv * kDK;
+    const long sbase = ((long)chunk_state_index(m, seq) * H + h) * (long)dv * kDK;
     float st[kDVS];
 #pragma unroll
     for (int vv = 0; vv < kDVS; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
@@ -620,8 +624,6 @@ gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
       unsigned char* stg = stage(s);
       const uint32_t a = smem_u32(stg);
       const float* gates = reinterpret_cast<const float*>(stg + S_PT + WS_G);
-      const int t0 = c * kC;
-      const int L = min(kC, T - t0);
       uint64_t* ready = reinterpret_cast<uint64_t*>(&cs.ready[s]);
       if (tid == 0 && !mbar_wait(ready, use & 1u, spin_limit)) give_up(ready, use & 1u, false);
       named_bar(1, 128);
@@ -765,19 +767,20 @@ uint32_t split_spin_limit() {
 }
 
 template <typename Tout>
-cudaError_t launch_split_t(const PrefillArgs& a, cudaStream_t stream) {
+cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
+  // packed sequences: the tensors are [1, total, H, *]
+  const int TB = m.cu ? 1 : a.B;
   CUtensorMap mq, mk, mv;
-  if (!encode_bthd_bf16(&mq, a.q, a.B, a.T, a.H, kDK, 64, kC, true) ||
-      !encode_bthd_bf16(&mk, a.k, a.B, a.T, a.H, kDK, 64, kC, true) ||
-      !encode_bthd_bf16(&mv, a.v, a.B, a.T, a.H, a.dv, kDVS, kC, false))
+  if (!encode_bthd_bf16(&mq, a.q, TB, a.T, a.H, kDK, 64, kC, true) ||
+      !encode_bthd_bf16(&mk, a.k, TB, a.T, a.H, kDK, 64, kC, true) ||
+      !encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, kDVS, kC, false))
     return cudaErrorInvalidValue;
-  const int nchunks = (a.T + kC - 1) / kC;
   const uint32_t lim = split_spin_limit();
   cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  gdn_chunk_prep_kernel<<<a.B * a.H * nchunks, P_THREADS, P_SMEM, stream>>>(
-      mq, mk, a.alpha, a.beta, (unsigned char*)a.workspace, a.T, a.H, nchunks,
+  gdn_chunk_prep_kernel<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
+      mq, mk, a.alpha, a.beta, (unsigned char*)a.workspace, m, a.H,
       (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -785,9 +788,9 @@ cudaError_t launch_split_t(const PrefillArgs& a, cudaStream_t stream) {
   auto carry = gdn_chunk_carry_kernel<Tout>;
   e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
   if (e != cudaSuccess) return e;
-  carry<<<a.B * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
-      mq, mk, mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, a.T, a.H,
-      a.dv, nchunks, (unsigned int*)a.workspace, lim);
+  carry<<<m.nseq * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
+      mq, mk, mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H,
+      a.dv, (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();
   if (e == cudaSuccess) timing_mark(stream, 1);
   return e;
@@ -800,9 +803,11 @@ size_t split_prefill_workspace(int B, int T, int H) {
   return (size_t)B * H * nchunks * kChunkWs;
 }
 
-cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream) {
-  if (a.out_dtype == GDR_F32) return launch_split_t<float>(a, stream);
-  return launch_split_t<__nv_bfloat16>(a, stream);
+size_t split_chunk_image_bytes() { return kChunkWs; }
+
+cudaError_t launch_prefill_split(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
+  if (a.out_dtype == GDR_F32) return launch_split_t<float>(a, m, stream);
+  return launch_split_t<__nv_bfloat16>(a, m, stream);
 }
 
 }  // namespace gdr

@@ -33,6 +33,7 @@
 #include <math.h>
 #include <stdlib.h>
 
+#include "chunkmap.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -620,11 +621,7 @@ bool tc_prefill_supported(const PrefillArgs& a) {
   return a.in_dtype == GDR_BF16 && a.dk == kDK && a.dv % kDVS == 0;
 }
 
-size_t split_prefill_workspace(int B, int T, int H);            // prefill_split.cu
-cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_kda_tc(const PrefillArgs& a, cudaStream_t stream);  // prefill_kda_tc.cu
-size_t kda_split_workspace(int B, int T, int H);                                // prefill_kda_split.cu
-cudaError_t launch_prefill_kda_split(const PrefillArgs& a, cudaStream_t stream);
 
 // The two-kernel paths (per-chunk prep over the whole GPU, then the carry) need a
 // workspace of 33 KB (GDN) or 128.5 KB (KDA) per chunk; with a smaller workspace the
@@ -640,11 +637,19 @@ size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
-  if (a.kda) {
-    if (a.ws_bytes >= 256 + kda_split_workspace(a.B, a.T, a.H)) return launch_prefill_kda_split(a, st);
-    return launch_prefill_kda_tc(a, st);
+  const bool split = a.ws_bytes >= 256 + (a.kda ? kda_split_workspace(a.B, a.T, a.H)
+                                                : split_prefill_workspace(a.B, a.T, a.H));
+  if (split) {
+    // dense batch: chunk gc of head h is chunk gc % nchunks of sequence gc / nchunks
+    ChunkMap m{};
+    m.nseq = a.B;
+    m.T = a.T;
+    m.nchunks = (a.T + GDR_CHUNK - 1) / GDR_CHUNK;
+    m.nck = a.B * m.nchunks;
+    m.img_base = 256;
+    return a.kda ? launch_prefill_kda_split(a, m, st) : launch_prefill_split(a, m, st);
   }
-  if (a.ws_bytes >= 256 + split_prefill_workspace(a.B, a.T, a.H)) return launch_prefill_split(a, st);
+  if (a.kda) return launch_prefill_kda_tc(a, st);
   if (a.out_dtype == GDR_F32) return launch_t<float>(a, st);
   return launch_t<__nv_bfloat16>(a, st);
 }

@@ -118,6 +118,45 @@ GDR_API gdr_status kda_prefill(const void* q, const void* k, const void* v,
                        int in_dtype, int out_dtype, int chunk,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* Packed variable-length prefill.  "Super Apriel: One Checkpoint, Many Speeds", §2D
+ * (inference and serving) and §4 (context-length scaling): a serving engine prefills
+ * prompts of many lengths together and keeps each one's recurrent state for its later
+ * decode steps.  nseq sequences are packed along the token axis:
+ *
+ *   q, k        [total, H, d_k]  bf16; sequence i is rows cu_seqlens[i] .. cu_seqlens[i+1]-1
+ *   v           [total, H, d_v]  bf16
+ *   alpha       GDN: [total, H] fp32;  KDA: [total, H, d_k] fp32
+ *   beta        [total, H] fp32
+ *   cu_seqlens  [nseq + 1] int32 DEVICE array, cu_seqlens[0] = 0, non-decreasing,
+ *               cu_seqlens[nseq] = total (a sequence may be empty)
+ *   state       [nslots, H, d_v, d_k] fp32 pool: sequence i starts from slot slots[i]
+ *               and its final state is written back there (in place); slots is an
+ *               int32 DEVICE array [nseq], or NULL for slot i; slots must be distinct
+ *   o           [total, H, d_v]  out_dtype (written)
+ *   workspace   gdr_prefill_varlen_workspace_bytes(...) bytes, 256-byte aligned,
+ *               zero-filled at allocation (the status word stays zero between calls)
+ *
+ * Chunks of 64 tokens never cross a sequence boundary.  Runs on the bf16 two-kernel
+ * tensor-core path only: in_dtype GDR_BF16, d_k = 128, d_v in {32, 64, 128}; other
+ * parameters return GDR_ERR_UNSUPPORTED.  Offsets that are not a partition of
+ * [0, total) are detected on the device: no chunk is processed and
+ * gdr_workspace_status returns GDR_ERR_INVALID_ARG. */
+GDR_API size_t gdr_prefill_varlen_workspace_bytes(int nseq, int total, int H, int dk, int dv,
+                                                  int kda);
+GDR_API gdr_status gdn_prefill_varlen(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const int* cu_seqlens,
+                       const int* slots, float* state, void* o,
+                       int nseq, int total, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream);
+/* Same contract as gdn_prefill_varlen with the per-channel gate alpha [total, H, d_k]. */
+GDR_API gdr_status kda_prefill_varlen(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const int* cu_seqlens,
+                       const int* slots, float* state, void* o,
+                       int nseq, int total, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream);
+
 /* One decode step: one new token for each of N sequences, the state updated IN
  * PLACE.
  *
@@ -204,7 +243,8 @@ GDR_API int gdr_prefill_path(int dk, int dv, int in_dtype, int kda);
 /* Synchronises `stream`, reads the device status word in `workspace` and clears
  * it.  Returns GDR_OK, GDR_ERR_TIMEOUT if a bounded device-side wait of a
  * prefill kernel gave up since the last check (the outputs of that call are
- * then undefined), or GDR_ERR_CUDA. */
+ * then undefined), GDR_ERR_INVALID_ARG if a packed-sequence call found its offsets
+ * inconsistent (nothing was processed), or GDR_ERR_CUDA. */
 GDR_API gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream);
 
 /* Measurement aid; the paper has no counterpart.  gdr_timing_start() clears the

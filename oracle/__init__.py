@@ -20,10 +20,11 @@ d_k-vector (KDA) in [0, 1], and beta_t a scalar.
 Modules
 -------
 recurrent   the definition, token by token (the oracle proper); decode_step and
-            verify_steps (K tokens with the state after each) run it from a state
+            verify_steps (K tokens with the state after each) run it from a state;
+            prefill_varlen runs packed sequences from a pool of state slots
 chunked     an independent fp64 chunk-wise restatement, used only to pin the
             chunk algebra against the definition
 """
 
-from .recurrent import gated_delta_rule, decode_step, verify_steps  # noqa: F401
+from .recurrent import gated_delta_rule, decode_step, verify_steps, prefill_varlen  # noqa: F401
 from .chunked import chunked_gated_delta_rule  # noqa: F401

@@ -114,3 +114,33 @@ def verify_steps(q, k, v, alpha, beta, state):
         outs.append(o[:, 0])
         snaps.append(S)
     return np.stack(outs, axis=1), np.stack(snaps, axis=0)
+
+
+def prefill_varlen(q, k, v, alpha, beta, cu_seqlens, state, slots=None):
+    """Sequences of different lengths packed along the token axis, each run from (and
+    back into) its own slot of a state pool.
+
+    "Super Apriel: One Checkpoint, Many Speeds", §2D (serving) and §4 (context-length
+    scaling): prompts of many lengths are prefilled together and each keeps its state.
+    Sequence i is tokens cu_seqlens[i] .. cu_seqlens[i+1]-1 and runs the recurrence
+    from state[slots[i]] (slot i when slots is None); nothing crosses a boundary.
+
+      q, k [total, H, d_k]; v [total, H, d_v]; alpha [total, H] or [total, H, d_k];
+      beta [total, H]; state [nslots, H, d_v, d_k] (not modified).
+    Returns (o [total, H, d_v], new_state [nslots, H, d_v, d_k]) in fp64.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    alpha, beta = _as_f64(alpha), _as_f64(beta)
+    cu = [int(x) for x in cu_seqlens]
+    pool = _as_f64(state).copy()
+    o = np.zeros(v.shape)
+    for i in range(len(cu) - 1):
+        a, b = cu[i], cu[i + 1]
+        slot = i if slots is None else int(slots[i])
+        if b == a:
+            continue
+        oi, si = gated_delta_rule(q[None, a:b], k[None, a:b], v[None, a:b], alpha[None, a:b],
+                                  beta[None, a:b], pool[slot][None])
+        o[a:b] = oi[0]
+        pool[slot] = si[0]
+    return o, pool

@@ -412,3 +412,68 @@ def test_verify_leaves_the_input_state():
     keep = S0.copy()
     verify_steps(q, k, v, alpha, beta, S0)
     assert np.array_equal(S0, keep)
+
+
+# --------------------------------------------------------------------------------------
+# prefill_varlen: packed sequences of different lengths with a pool of state slots
+
+from oracle import prefill_varlen  # noqa: E402
+
+
+def _varlen_case(kda, lens, H=2, dk=4, dv=3, nslots=None, seed=41):
+    rng = np.random.default_rng(seed)
+    total = sum(lens)
+    q = rng.standard_normal((total, H, dk))
+    k = rng.standard_normal((total, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((total, H, dv))
+    alpha = rng.uniform(0.2, 1.0, size=(total, H, dk) if kda else (total, H))
+    beta = rng.uniform(0.1, 1.0, size=(total, H))
+    pool = rng.standard_normal((nslots or len(lens), H, dv, dk))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return q, k, v, alpha, beta, cu, pool
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_varlen_equal_lengths_is_the_batched_call(kda):
+    """nseq sequences of T tokens each, slot i: the same as one [nseq, T] batch."""
+    q, k, v, alpha, beta, cu, pool = _varlen_case(kda, [5, 5, 5])
+    o, new = prefill_varlen(q, k, v, alpha, beta, cu, pool)
+    sh = lambda x: x.reshape((3, 5) + x.shape[1:])  # noqa: E731
+    ob, sb = gated_delta_rule(sh(q), sh(k), sh(v), sh(alpha), sh(beta), pool)
+    assert np.allclose(o, ob.reshape(o.shape), rtol=1e-14, atol=1e-14)
+    assert np.allclose(new, sb, rtol=1e-14, atol=1e-14)
+
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_varlen_ragged_matches_the_chunked_restatement(kda):
+    """Ragged lengths (including an empty sequence) and permuted slots, against the
+    independent chunk-wise code run sequence by sequence."""
+    lens = [7, 0, 1, 12, 4]
+    slots = [5, 0, 2, 1, 3]
+    q, k, v, alpha, beta, cu, pool = _varlen_case(kda, lens, nslots=7, seed=42)
+    o, new = prefill_varlen(q, k, v, alpha, beta, cu, pool, slots)
+    for i, (a, b) in enumerate(zip(cu[:-1], cu[1:])):
+        s = slots[i]
+        if a == b:
+            assert np.array_equal(new[s], pool[s])
+            continue
+        oc, sc = chunked_gated_delta_rule(q[None, a:b], k[None, a:b], v[None, a:b],
+                                          alpha[None, a:b], beta[None, a:b], pool[s][None],
+                                          chunk=4)
+        assert np.allclose(o[a:b], oc[0], rtol=1e-12, atol=1e-12)
+        assert np.allclose(new[s], sc[0], rtol=1e-12, atol=1e-12)
+    for s in (4, 6):                       # slots no sequence uses are left alone
+        assert np.array_equal(new[s], pool[s])
+
+
+def test_varlen_sequences_do_not_leak_into_each_other():
+    """Changing one sequence's tokens changes no other sequence's outputs or state."""
+    q, k, v, alpha, beta, cu, pool = _varlen_case(True, [6, 9, 3], seed=43)
+    o1, s1 = prefill_varlen(q, k, v, alpha, beta, cu, pool)
+    v2 = v.copy()
+    v2[6:15] += 1.0                        # sequence 1 only
+    o2, s2 = prefill_varlen(q, k, v2, alpha, beta, cu, pool)
+    assert np.array_equal(o1[:6], o2[:6]) and np.array_equal(o1[15:], o2[15:])
+    assert np.array_equal(s1[0], s2[0]) and np.array_equal(s1[2], s2[2])
+    assert not np.allclose(s1[1], s2[1])
