@@ -27,12 +27,13 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, device_inputs, slice_inputs  # noqa: E402
+from synth import WORKLOADS, device_inputs, slice_inputs, tokens, varlen_lengths  # noqa: E402
 
 METRIC = "GDN/KDA prefill tokens/s and decode tokens/s at 1 B200; % of roofline"
 L2_BYTES = 126 * 2 ** 20
@@ -50,7 +51,7 @@ def algorithmic(w):
     triangular solve and the gate exponentials).  Decode counts the state bytes
     (read + write) only, which is 99% of its traffic."""
     esz = 2 if w.dtype == "bf16" else 4
-    th = w.B * w.T * w.H
+    th = tokens(w) * w.H
     state = w.B * w.H * w.dv * w.dk * 4
     if w.decode:
         return 2 * state * w.T, th * 6 * w.dk * w.dv
@@ -62,6 +63,7 @@ def algorithmic(w):
         return (1 + w.T) * state + th * per_th, th * 6 * w.dk * w.dv
     a_bytes = 4 * (w.dk if w.mixer == "kda" else 1)
     per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
+    # the final states are written; initial states read when the workload has them
     nbytes = th * per_th + state + (state if w.state == "randn" else 0)
     C = 64
     flops = th * (2 * C * (3 * w.dk + 2 * w.dv) + 6 * w.dk * w.dv)
@@ -288,6 +290,40 @@ class VerifyRunner:
                 o=self.o)
 
 
+class VarlenRunner:
+    """One packed prefill call per step: B prompts of varlen_lengths(w) tokens, each
+    from and back into its own slot of a state pool (inputs > 3x L2)."""
+
+    def __init__(self, w, dev, seed):
+        import gated_delta_rule_79_b200 as g
+        self.g, self.w, self.dev = g, w, dev
+        self.fn = g.kda_prefill_varlen if w.mixer == "kda" else g.gdn_prefill_varlen
+        lens = varlen_lengths(w)
+        total = sum(lens)
+        x = device_inputs(w.with_(B=1, T=total, varlen=False), dev, seed=seed)
+        self.x = {k: (v[0] if k != "s0" else None) for k, v in x.items()}
+        gen = torch.Generator(device=dev).manual_seed(seed + 1)
+        self.pool = 0.02 * torch.randn((w.B, w.H, w.dv, w.dk), generator=gen, device=dev)
+        self.cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=dev)
+        self.o = torch.empty((total, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        need = g.lib.gdr_prefill_varlen_workspace_bytes(w.B, total, w.H, w.dk, w.dv,
+                                                        int(w.mixer == "kda"))
+        self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        self.kernels = ["varlen index + " + f"{w.mixer}_chunk_prep_kernel",
+                        f"{w.mixer}_chunk_carry_kernel"]
+        self.launches_per_step = 3
+        self.kernel_key = f"prefill_two-kernel:{w.name}"
+        self.path = "tensor-core"
+        in_bytes = sum(t.numel() * t.element_size() for t in self.x.values() if t is not None)
+        self.l2_note = (f"{len(lens)} prompts, {total} tokens, {in_bytes / 2**20:.0f} MiB of "
+                        f"inputs (> 3x L2)")
+
+    def step(self, i):
+        x = self.x
+        self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], self.cu, self.pool, o=self.o,
+                workspace=self.ws)
+
+
 def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
     """Warm up, then time exactly `steps` steps with CUDA events on the launching
     stream, bracketed by a barrier and a synchronize on both sides.  Also records
@@ -351,6 +387,30 @@ def time_e2e(w, dev, steps, warmup, seed):
                     dbuf[key].copy_(host[key][t], non_blocking=True)
                 fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o)
                 o_host[t].copy_(o, non_blocking=True)
+    elif w.varlen:
+        fn = g.kda_prefill_varlen if w.mixer == "kda" else g.gdn_prefill_varlen
+        lens = varlen_lengths(w)
+        total = sum(lens)
+        xd = device_inputs(w.with_(B=1, T=total, varlen=False), dev, seed=seed + 100)
+        keys = ("q", "k", "v", "alpha", "beta")
+        host = {k: xd[k][0].cpu().pin_memory() for k in keys}
+        dbuf = {k: torch.empty_like(xd[k][0]) for k in keys}
+        pool = 0.02 * torch.randn((w.B, w.H, w.dv, w.dk), device=dev)
+        cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=dev)
+        o = torch.empty((total, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        need = g.lib.gdr_prefill_varlen_workspace_bytes(w.B, total, w.H, w.dk, w.dv,
+                                                        int(w.mixer == "kda"))
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = o.numel() * 2
+
+        def step():
+            for key in keys:
+                dbuf[key].copy_(host[key], non_blocking=True)
+            fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], cu, pool, o=o,
+               workspace=ws)
+            o_host.copy_(o, non_blocking=True)
     elif w.verify:
         fn = g.kda_verify if w.mixer == "kda" else g.gdn_verify
         keys = ("q", "k", "v", "alpha", "beta")
@@ -396,7 +456,7 @@ def time_e2e(w, dev, steps, warmup, seed):
     b.record(stream)
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / steps
-    return {"value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+    return {"value": tokens(w) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
 
 
@@ -503,7 +563,7 @@ def main():
         v = statistics.median(rates)
         cores, sample = ot.cores, ot.sample
         line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": a.gpus,
-                "steps": steps, "warmup": warmup, "ms_per_step": w.B * w.T / v * 1e3,
+                "steps": steps, "warmup": warmup, "ms_per_step": tokens(w) / v * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic", "impl": "reference",
                 "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
@@ -522,15 +582,15 @@ def main():
     active = dist_init(world, "nccl")
     peaks, peak_kind = load_peaks()
     runner = (DecodeRunner if w.decode else VerifyRunner if w.verify
-              else PrefillRunner)(w, dev, seed=1000 * rank)
+              else VarlenRunner if w.varlen else PrefillRunner)(w, dev, seed=1000 * rank)
     clocks = ClockSampler(dev.index)
     clocks.start()
     total_ms, per, kernel_ms = time_device(runner, steps, warmup, dev, active)
     clk = clocks.stop()
     ms_step = total_ms / steps
     max_ms = max_over_ranks(total_ms, active, dev)
-    tokens = w.B * w.T
-    value = aggregate(tokens * steps, max_ms, world)
+    ntok = tokens(w)
+    value = aggregate(ntok * steps, max_ms, world)
     nbytes, flops = algorithmic(w)
     kern_ms = statistics.mean(per)
     if w.decode:
@@ -570,7 +630,8 @@ def main():
             "dtype": "bf16" if runner.path == "tensor-core" else "f32",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                       "in_dtype": w.dtype, "out_dtype": "bf16", "chunk": 64,
+                       "tokens_per_step": ntok, "in_dtype": w.dtype, "out_dtype": "bf16",
+                       "chunk": 64,
                        "kernel": runner.path, "l2": runner.l2_note,
                        "clocks_window": "0.5 s soak of the same steps, then the timed region",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},

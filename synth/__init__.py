@@ -14,6 +14,8 @@ Workloads (all inputs synthetic; the pages publish no dataset for the mixer):
   kda_long      KDA, B=4 H=32 T=65536 d=128, bf16, state ~ 0.02 N(0,1)
   verify_gdn    N=256 sequences x H=32, d=128, K=4 tokens from a carried state
   verify_kda    ~ 0.02 N(0,1), bf16 q/k/v; GDN and KDA gates (B = N, T = K)
+  gdn_varlen    64 prompts packed along the tokens, H=32, d=128, bf16, each from its
+  kda_varlen    own slot of a state pool ~ 0.02 N(0,1); lengths from varlen_lengths
 
 Recipe per (batch b, head h) slice, one ``torch.Generator`` (CPU) seeded with
 ``slice_seed(seed, b, h)``, drawing in this fixed order:
@@ -53,6 +55,7 @@ class Workload:
     state: str          # "zeros" or "randn"
     decode: bool = False
     verify: bool = False  # K tokens (the T axis) from a carried state, snapshots kept
+    varlen: bool = False  # B sequences of varlen_lengths(w) tokens packed (T: median)
 
     @property
     def torch_dtype(self):
@@ -73,7 +76,20 @@ WORKLOADS = {
                            verify=True),
     "verify_kda": Workload("verify_kda", "kda", 256, 32, 4, 128, 128, "bf16", "randn",
                            verify=True),
+    "gdn_varlen": Workload("gdn_varlen", "gdn", 64, 32, 256, 128, 128, "bf16", "randn",
+                           varlen=True),
+    "kda_varlen": Workload("kda_varlen", "kda", 64, 32, 256, 128, 128, "bf16", "randn",
+                           varlen=True),
 }
+
+
+def varlen_lengths(w: Workload, seed: int = 0):
+    """Prompt lengths of a packed workload: log-normal around the median w.T
+    (sigma 0.8), rounded, clipped to [1, 16 w.T], drawn from a seeded CPU generator."""
+    g = torch.Generator().manual_seed(1_000_003 * seed + 17)
+    x = torch.randn(w.B, generator=g, dtype=torch.float64)
+    lens = torch.exp(math.log(w.T) + 0.8 * x).round().clamp(1, 16 * w.T).to(torch.int64)
+    return [int(n) for n in lens]
 
 
 def slice_seed(seed, b, h):
@@ -169,7 +185,10 @@ def device_inputs(w: Workload, device, seed: int = 0, dtype_override=None):
 
 
 def tokens(w: Workload):
-    """Tokens processed by one pass of the workload (prefill: B*T; decode: N*steps)."""
+    """Tokens processed by one pass of the workload (prefill: B*T; decode: N*steps;
+    packed: the sum of the lengths)."""
+    if w.varlen:
+        return sum(varlen_lengths(w))
     return w.B * w.T
 
 

@@ -197,3 +197,14 @@ def test_in_place_state_carry(mixer):
     torch.cuda.synchronize()
     assert s.data_ptr() == state.data_ptr()
     check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], "alias")
+
+
+@pytest.mark.parametrize("dv", [128, 64])
+def test_kda_carry_with_64_value_columns(dv):
+    """With enough (sequence, head) chains the KDA carry takes 64 value columns per CTA
+    (two slices sharing each chunk's operands): 3 x 50 heads run that way."""
+    w = Workload("wide", "kda", 3, 50, 130, 128, dv, "bf16", "randn")
+    x = make_inputs(w, seed=77)
+    o, s = gpu_prefill("kda", x, out_dtype=torch.float32)
+    o_ref, s_ref = ref_prefill(x)
+    check(o, s, o_ref, s_ref, TOL["bf16"], f"kda 64-column carry dv={dv}")
