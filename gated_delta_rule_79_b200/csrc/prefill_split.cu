@@ -10,26 +10,23 @@
 //   O = Diag(e^G) Q S0^T + P U
 //   S^T <- e^{G_last} S0^T + K^T Diag(e^{G_last-G}) U
 //
-// P, T and the gate factors do not depend on the state, so gdn_chunk_prep_kernel
-// computes them for every chunk of every head at once (the whole GPU works on
-// them in parallel) and leaves them in the workspace as operand tiles ready to be
-// copied; gdn_chunk_carry_kernel then walks the chunks of each (head, 32-wide
-// value slice) and only runs the state-dependent products.  Its loader warpgroup
-// brings chunk c+1 in (TMA for q, k, v; a bulk copy for P, T, gates) and builds
-// k^T while the carry warpgroup works on chunk c.
+// Everything but the state-dependent products is computed by gdn_chunk_prep_kernel
+// for every chunk of every head at once (the whole GPU works on them in parallel):
+// the Gram [Q; K] K^T runs as one exact kind::f16 product on the bf16 q, k tiles (the
+// scalar decays e^{G_t - G_j} are applied on read-back), then the triangular solve
+// gives T.  It leaves the chunk's operand images for the carry in the workspace
+// (chunk_image.cuh): [Q (.) e^G; K (.) e^G], e^{G_last}, T, (K (.) e^{G_last - G})^T and
+// P as tf32 tiles.  The state carry that walks the chunks in order is shared with KDA
+// (carry.cu).
 //
-// Precision: q, k, v are bf16 and exact; products with them run as kind::f16 with
-// the computed partner (the state, Diag(e^{G_last-G}) U) split into bf16 hi + lo
-// (about 16 significant bits).  Products of two computed operands (T R, P U) run
-// as kind::tf32 with operands rounded to nearest.  Measured by emulation, single
-// bf16 roundings cost about 3e-3 normwise error against a 2e-3 budget.
-//
-// Waits are bounded; a give-up records GDR_ERR_TIMEOUT in the workspace status
-// word, drains what was issued, frees tensor memory and ends the CTA.
+// Precision: the Gram is exact (bf16 inputs, fp32 accumulation); the carry's products
+// run as kind::tf32 with operands rounded to nearest.  Waits are bounded; a give-up
+// records GDR_ERR_TIMEOUT in the workspace status word and ends the CTA.
 
 #include <math.h>
 #include <stdlib.h>
 
+#include "chunk_image.cuh"
 #include "chunkmap.cuh"
 #include "common.cuh"
 #include "launch.h"
@@ -46,9 +43,8 @@ constexpr int kDK = 128;
 constexpr int kDVS = 32;
 constexpr uint32_t kDrainLimit = 1u << 26;
 
-// Workspace per chunk: P tile (fp32, 16 KB) | T tile (16 KB) | gates (1 KB:
-// e^{G_t}[64], e^{G_last - G_t}[64], e^{G_last}).
-constexpr int kChunkWs = 33792;
+// The prep's shared-memory staging of P | T | gate factors (e^{G_t}[64],
+// e^{G_last - G_t}[64], e^{G_last}); P and T are copied to the chunk image from here.
 constexpr int WS_T = 16384, WS_G = 32768;
 constexpr size_t kStatusBytes = 256;
 
@@ -88,7 +84,7 @@ constexpr int P_QK = 0;                    // bf16 [128][128] SW128 (q rows 0-63
 constexpr int P_X = 0;                     //   X scratch, sx() layout                        16 KB
 constexpr int P_A = 16384;                 //   packed strictly-lower A                       10 KB
 constexpr int P_Z = P_A + 10240;           //   level scratch [3][16][16]                      3 KB
-constexpr int P_OUT = 32768;               // P | T | gates: the chunk's workspace image      33 KB
+constexpr int P_OUT = 32768;               // P | T | gates (staging)                         33 KB
 constexpr int P_SMALL = P_OUT + 34816;
 constexpr int P_SMEM = P_SMALL + 1024 + 1024;   // 68 KB: three CTAs per SM
 constexpr uint32_t P_TM_COLS = 64;
@@ -196,6 +192,45 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int ks = 0; ks < kDK / 16; ++ks)
       mma_bf16_w(tb, kstep(dA, 128, ks), kstep(dB, 128, ks), id, ks > 0);
     mma_commit_w(mma_bar);
+  }
+  // ---- while the Gram runs: the carry's images of this chunk (chunk_image.cuh), from the
+  //      q/k tile (which the solve's scratch overwrites later): [Q (.) e^G; K (.) e^G], e^{G_last},
+  //      K^ = (K (.) e^{G_last - G})^T (tokens past L: zero)
+  unsigned char* img = ws + m.img_base + ((size_t)h * m.nck + gc) * img::kChunkWs;
+  {
+    // Each warp store writes four whole 128-byte tile rows: lane l takes 16-byte chunk
+    // l % 8 of row 4 i + l / 8 of a panel (4 tf32 channels, or 4 tokens for K^).
+    const int sub = lane >> 3, cd = lane & 7;
+    // [Q~; K~]: 128 rows x 4 panels of 32 channels
+#pragma unroll 4
+    for (int it = 0; it < 32; ++it) {
+      const int unit = it * 4 + warp;                 // 0..127: (row group, panel)
+      const int pd = unit & 3, r = 4 * (unit >> 2) + sub;
+      const int ch = 32 * pd + 4 * cd;                // first of the 4 channels
+      const uint2 x = *reinterpret_cast<const uint2*>(
+          tQK + (ch >> 6) * 16384 + r * 128 + ((((ch & 63) >> 3) ^ (r & 7)) << 4) + ((ch & 7) << 1));
+      const float eg = gates[r & 63];
+      *reinterpret_cast<float4*>(img + img::WS_QK + pd * 16384 + r * 128 + ((cd ^ (r & 7)) << 4)) =
+          img::tf32x4(__uint_as_float(x.x << 16) * eg, __uint_as_float(x.x & 0xffff0000u) * eg,
+                      __uint_as_float(x.y << 16) * eg, __uint_as_float(x.y & 0xffff0000u) * eg);
+    }
+    reinterpret_cast<float*>(img + img::WS_EGL)[tid] = gates[128];
+    // K^: 128 rows (channels) x 2 panels of 32 tokens; tokens past L are zero
+#pragma unroll 4
+    for (int it = 0; it < 16; ++it) {
+      const int unit = it * 4 + warp;                 // 0..63: (row group, panel)
+      const int pd = unit & 1, c = 4 * (unit >> 1) + sub;
+      float f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = 32 * pd + 4 * cd + u;
+        const float kv = __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(tQK + swz_off_bf16(64 + j, c, 128)));
+        f[u] = j < L ? kv * gates[64 + j] : 0.f;
+      }
+      *reinterpret_cast<float4*>(img + img::WS_KH + pd * 16384 + c * 128 + ((cd ^ (c & 7)) << 4)) =
+          img::tf32x4(f[0], f[1], f[2], f[3]);
+    }
   }
   if (!mbar_wait(mma_bar, 0, spin_limit)) {
     mbar_wait(mma_bar, 0, kDrainLimit);
@@ -344,420 +379,11 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   fence_smem_to_async();
   __syncthreads();
   if (tid == 0) {
-    unsigned char* dst = ws + m.img_base + ((size_t)h * m.nck + gc) * kChunkWs;
-    bulk_store(dst, smem_u32(tP), kChunkWs);
+    bulk_store(img + img::WS_P, smem_u32(tP), 16384);
+    bulk_store(img + img::WS_T, smem_u32(tT), 16384);
     bulk_commit();
     bulk_wait_all();
   }
-}
-
-// ========================================================================================
-// Kernel 2: the state carry, per (batch, head, 32-wide slice of d_v)
-// ========================================================================================
-
-constexpr int C_THREADS = 256;             // warps 0-3 carry, warps 4-7 load
-constexpr int C_STAGES = 2;
-// one stage (bytes from the stage base)
-constexpr int S_QK = 0;                    // bf16 [128][128] SW128 (TMA)                  32 KB
-constexpr int S_KT = 32768;                // bf16 [128 c][64 j] SW128 k^T                 16 KB
-constexpr int S_PT = 49152;                // P | T | gates (bulk copy of the workspace)   33 KB
-constexpr int S_V = S_PT + 34816;          // bf16 [64 j][32 v] (TMA)                       4 KB
-constexpr int STAGE_BYTES = S_V + 4096;    // 88 KB
-constexpr uint32_t STAGE_TX = 32768 + 4096 + kChunkWs;
-// carry-side tiles
-constexpr int C_SSH = C_STAGES * STAGE_BYTES;   // bf16 [32 v][128 c] state hi           8 KB
-constexpr int C_SSL = C_SSH + 8192;             // state lo                               8 KB
-constexpr int C_RT = C_SSL + 8192;              // fp32 [32 v][64 j]; P U exchange        8 KB
-constexpr int C_UT = C_RT + 8192;               // fp32 [32 v][64 j]                      8 KB
-constexpr int C_UPH = C_UT + 8192;              // bf16 [32 v][64 j] (e^{G_last-G} U) hi  4 KB
-constexpr int C_UPL = C_UPH + 4096;             //                                  lo    4 KB
-constexpr int C_OX = C_UPL + 4096;              // P U exchange [64 t][32 v] (loader)    8 KB
-constexpr int C_SMALL = C_OX + 8192;
-constexpr int C_SMEM = C_SMALL + 1024 + 1024;
-static_assert(C_SMEM <= 232448, "shared memory");
-
-// [q; k] S0^T (M=128 x 32: rows 0-63 O1, rows 64-127 Y) and P U (M=64 x 32) are
-// double-buffered by chunk parity: the loader warpgroup reads chunk c's outputs while
-// the carry already runs chunk c+1.
-constexpr uint32_t TM_OY = 0;    // + 32 * (c & 1)
-constexpr uint32_t TM_O2 = 64;   // + 32 * (c & 1)
-constexpr uint32_t TM_U = 128;   // U, M=64 x 32
-constexpr uint32_t TM_S = 160;   // S^T, M=128 x 32
-constexpr uint32_t C_TM_COLS = 256;
-
-struct CarrySmall {
-  unsigned long long full[C_STAGES];    // TMA + bulk copy landed
-  unsigned long long ready[C_STAGES];   // k^T built, stage ready for the carry
-  unsigned long long empty[C_STAGES];   // carry done with the stage
-  unsigned long long mma_bar;
-  unsigned long long out_full[2];   // chunk's O1 and P U are in TMEM (carry -> loader)
-  unsigned long long out_empty[2];  // loader has read them (loader -> carry)
-  float eg_out[2][64];              // e^{G_t} of the chunk whose outputs are pending
-  uint32_t tmem;
-  int abort;
-};
-
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(x);
-  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
-
-template <typename Tout>
-__global__ void __launch_bounds__(C_THREADS, 1)
-gdn_chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v,
-                       const unsigned char* __restrict__ ws, const float* __restrict__ s0,
-                       Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m,
-                       int H, int dv, unsigned int* __restrict__ status, uint32_t spin_limit) {
-  extern __shared__ unsigned char smem_raw[];
-  const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  unsigned char* sm = smem_raw + padb;
-  CarrySmall& cs = *reinterpret_cast<CarrySmall*>(sm + C_SMALL);
-  unsigned char* tSSH = sm + C_SSH;
-  unsigned char* tSSL = sm + C_SSL;
-  unsigned char* tRT = sm + C_RT;
-  unsigned char* tUT = sm + C_UT;
-  unsigned char* tUPH = sm + C_UPH;
-  unsigned char* tUPL = sm + C_UPL;
-  float* Ox = reinterpret_cast<float*>(sm + C_OX);   // P U exchange [64 t][32 v], row-XOR
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3;
-  const int nslice = dv / kDVS;
-  const int slice = blockIdx.x % nslice;
-  const int sh = blockIdx.x / nslice;
-  const int h = sh % H, seq = sh / H;
-  int first = 0, nchunks = 0;
-  chunk_range(m, seq, first, nchunks);
-  const int v0 = slice * kDVS;
-
-  if (tid == 0) {
-    for (int s = 0; s < C_STAGES; ++s) {
-      mbar_init(reinterpret_cast<uint64_t*>(&cs.full[s]), 1);
-      mbar_init(reinterpret_cast<uint64_t*>(&cs.ready[s]), 1);
-      mbar_init(reinterpret_cast<uint64_t*>(&cs.empty[s]), 1);
-    }
-    mbar_init(reinterpret_cast<uint64_t*>(&cs.mma_bar), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_full[s]), 1);
-      mbar_init(reinterpret_cast<uint64_t*>(&cs.out_empty[s]), 1);
-    }
-    cs.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(&cs.tmem, C_TM_COLS);
-  fence_before_sync();
-  __syncthreads();
-  fence_after_sync();
-  const uint32_t tb = cs.tmem;
-  const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
-  const unsigned char* wsb = ws + m.img_base + ((size_t)h * m.nck + first) * kChunkWs;
-
-  auto stage = [&](int s) { return sm + s * STAGE_BYTES; };
-  // A wait gave up: record the timeout and stop both warpgroups.  For barriers fed by
-  // the tensor cores or the copy engines, first drain what was issued (drain = true);
-  // the barriers between the two warpgroups have nothing to drain.
-  auto give_up = [&](uint64_t* bar, uint32_t parity, bool drain) {
-    if (drain) mbar_wait(bar, parity, kDrainLimit);
-    atomicOr(status, 1u);
-    cs.abort = 1;
-  };
-
-  if (warp >= 4) {
-    // =========================== loader warpgroup =====================================
-    const int lt = tid - 128;
-    // O = Diag(e^G) O1 + P U for chunk cc, read from the chunk's TMEM buffers once the
-    // carry has finished it; returns false on abort.
-    auto write_outputs = [&](int cc) -> bool {
-      const int ob = cc & 1;
-      const uint32_t use = (uint32_t)(cc >> 1);
-      uint64_t* ofull = reinterpret_cast<uint64_t*>(&cs.out_full[ob]);
-      if (lt == 0 && !mbar_wait(ofull, use & 1u, spin_limit)) give_up(ofull, use & 1u, false);
-      named_bar(2, 128);
-      if (cs.abort) return false;
-      fence_after_sync();
-      const ChunkLoc loc = chunk_locate(m, first + cc);
-      const int t0 = loc.t0, L = loc.L, b = loc.b;
-      {
-        float o2[32];
-        tmem_ld32(tb + tlane + TM_O2 + 32 * ob, o2);
-        tmem_wait_ld();
-        if (lane < 16) {
-          const int t = 16 * q4 + lane;
-#pragma unroll
-          for (int x = 0; x < 32; ++x) Ox[t * 32 + (x ^ (t & 31))] = o2[x];
-        }
-      }
-      named_bar(2, 128);
-      if (q4 < 2) {
-        const int t = 32 * q4 + lane;
-        float o1[32], o2[32];
-        tmem_ld32(tb + tlane + TM_OY + 32 * ob, o1);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) o2[x] = Ox[t * 32 + (x ^ (t & 31))];
-        const float eg = cs.eg_out[ob][t];
-        tmem_wait_ld();
-        if (t < L) {
-          Tout* dst = o + (((long)b * m.T + t0 + t) * H + h) * (long)dv + v0;
-          if constexpr (sizeof(Tout) == 2) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 pk;
-              __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&pk);
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                hp[x] = __floats2bfloat162_rn(fmaf(eg, o1[8 * q + 2 * x], o2[8 * q + 2 * x]),
-                                              fmaf(eg, o1[8 * q + 2 * x + 1], o2[8 * q + 2 * x + 1]));
-              reinterpret_cast<uint4*>(dst)[q] = pk;
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<float4*>(dst)[q] =
-                  make_float4(fmaf(eg, o1[4 * q], o2[4 * q]), fmaf(eg, o1[4 * q + 1], o2[4 * q + 1]),
-                              fmaf(eg, o1[4 * q + 2], o2[4 * q + 2]),
-                              fmaf(eg, o1[4 * q + 3], o2[4 * q + 3]));
-          }
-        }
-      }
-      fence_before_sync();
-      named_bar(2, 128);
-      if (lt == 0) mbar_arrive(reinterpret_cast<uint64_t*>(&cs.out_empty[ob]));
-      return true;
-    };
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1;
-      const uint32_t use = (uint32_t)(c >> 1);
-      unsigned char* st = stage(s);
-      uint64_t* full = reinterpret_cast<uint64_t*>(&cs.full[s]);
-      uint64_t* empty = reinterpret_cast<uint64_t*>(&cs.empty[s]);
-      uint64_t* ready = reinterpret_cast<uint64_t*>(&cs.ready[s]);
-      // wait until the carry has released this stage (first use passes at once)
-      bool ok = true;
-      if (lt == 0) {
-        if (!mbar_wait(empty, (use & 1u) ^ 1u, spin_limit)) {
-          give_up(empty, (use & 1u) ^ 1u, false);
-          ok = false;
-        }
-      }
-      named_bar(2, 128);
-      if (cs.abort) break;
-      if (lt == 0 && ok) {
-        const uint32_t a = smem_u32(st);
-        const ChunkLoc loc = chunk_locate(m, first + c);
-        const int t0 = loc.t0, b = loc.b;
-        mbar_expect_tx(full, STAGE_TX);
-        tma_load_4d(a + S_QK, &tm_q, 0, h, t0, b, full);
-        tma_load_4d(a + S_QK + 16384, &tm_q, 64, h, t0, b, full);
-        tma_load_4d(a + S_QK + 8192, &tm_k, 0, h, t0, b, full);
-        tma_load_4d(a + S_QK + 16384 + 8192, &tm_k, 64, h, t0, b, full);
-        tma_load_4d(a + S_V, &tm_v, v0, h, t0, b, full);
-        bulk_load(a + S_PT, wsb + (size_t)c * kChunkWs, kChunkWs, full);
-      }
-      if (!mbar_wait(full, use & 1u, spin_limit)) give_up(full, use & 1u, true);
-      named_bar(2, 128);
-      if (cs.abort) break;
-      // the loader forms this chunk's outputs later: keep its e^{G_t}
-      if (lt < 64) cs.eg_out[s][lt] = reinterpret_cast<const float*>(st + S_PT + WS_G)[lt];
-      // k^T: thread lt takes channel lt of every token of the chunk
-      {
-        const unsigned char* qk = st + S_QK;
-        unsigned char* kt = st + S_KT;
-        __nv_bfloat16 col[64];
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-          col[j] = *reinterpret_cast<const __nv_bfloat16*>(qk + swz_off_bf16(64 + j, lt, 128));
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 pk;
-          __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&pk);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) e[x] = col[8 * q + x];
-          *reinterpret_cast<uint4*>(kt + lt * 128 + ((q ^ (lt & 7)) << 4)) = pk;
-        }
-      }
-      fence_smem_to_async();
-      named_bar(2, 128);
-      if (lt == 0) mbar_arrive(ready);
-      if (c > 0 && !write_outputs(c - 1)) break;
-    }
-    if (!cs.abort && nchunks > 0) write_outputs(nchunks - 1);
-  } else {
-    // =========================== carry warpgroup ======================================
-    // state: thread c < 128 owns row c of S^T (S[v0 + v][c], v < 32)
-    const long sbase = ((long)chunk_state_index(m, seq) * H + h) * (long)dv * kDK;
-    float st[kDVS];
-#pragma unroll
-    for (int vv = 0; vv < kDVS; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
-    auto write_state_operand = [&]() {
-#pragma unroll
-      for (int vv = 0; vv < kDVS; ++vv) {
-        __nv_bfloat16 hi, lo;
-        split_bf16(st[vv], hi, lo);
-        const uint32_t off = swz_off_bf16(vv, tid, kDVS);
-        *reinterpret_cast<__nv_bfloat16*>(tSSH + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(tSSL + off) = lo;
-      }
-    };
-    write_state_operand();
-    fence_smem_to_async();
-    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&cs.mma_bar);
-    uint32_t mphase = 0;
-    const uint32_t aSSH = smem_u32(tSSH), aSSL = smem_u32(tSSL), aRT = smem_u32(tRT);
-    const uint32_t aUT = smem_u32(tUT), aUPH = smem_u32(tUPH), aUPL = smem_u32(tUPL);
-    const uint64_t dSSH = sdesc(aSSH, 16, 1024), dSSL = sdesc(aSSL, 16, 1024);
-    const uint64_t dRT = sdesc(aRT, 16, 1024), dUT = sdesc(aUT, 16, 1024);
-    const uint64_t dUPH = sdesc(aUPH, 16, 1024), dUPL = sdesc(aUPL, 16, 1024);
-    // bounded wait on the carry's MMA barrier; the result is the same in all 128 threads
-    auto wait_mma = [&]() -> bool {
-      if (!mbar_wait(mma_bar, mphase, spin_limit)) give_up(mma_bar, mphase, true);
-      mphase ^= 1u;
-      fence_after_sync();
-      named_bar(1, 128);
-      return cs.abort != 0;
-    };
-    bool aborted = false;
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1;
-      const uint32_t use = (uint32_t)(c >> 1);
-      unsigned char* stg = stage(s);
-      const uint32_t a = smem_u32(stg);
-      const float* gates = reinterpret_cast<const float*>(stg + S_PT + WS_G);
-      uint64_t* ready = reinterpret_cast<uint64_t*>(&cs.ready[s]);
-      if (tid == 0 && !mbar_wait(ready, use & 1u, spin_limit)) give_up(ready, use & 1u, false);
-      named_bar(1, 128);
-      if ((aborted = cs.abort != 0)) break;
-      fence_after_sync();
-      // ---- decay the state in TMEM, then [O1; Y] = [Q; K] (S_hi + S_lo)^T ----------------
-      const int ob = c & 1;
-      if (c >= 2 && tid == 0) {
-        uint64_t* oe = reinterpret_cast<uint64_t*>(&cs.out_empty[ob]);
-        const uint32_t par = (uint32_t)((c >> 1) - 1) & 1u;
-        if (!mbar_wait(oe, par, spin_limit)) give_up(oe, par, false);
-      }
-      {
-        float sd[kDVS];
-        const float egc = gates[128];
-#pragma unroll
-        for (int vv = 0; vv < kDVS; ++vv) sd[vv] = st[vv] * egc;
-        tmem_st32(tb + tlane + TM_S, sd);
-        tmem_wait_st();
-      }
-      fence_before_sync();
-      named_bar(1, 128);
-      if (warp == 0) {
-        fence_after_sync();
-        const uint64_t dQK = sdesc(a + S_QK, 16, 1024);
-        const uint32_t id = idesc_bf16(128, 32);
-#pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSH, kDVS, ks), id, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks)
-          mma_bf16_w(tb + TM_OY + 32 * ob, kstep(dQK, 128, ks), kstep(dSSL, kDVS, ks), id, true);
-        mma_commit_w(mma_bar);
-      }
-      if ((aborted = wait_mma())) break;
-      // ---- R = V - Diag(e^G) Y as the operand [v][j] (Y rows: TMEM lanes 64-127) ----------
-      if (q4 >= 2) {
-        const int j = 32 * (q4 - 2) + lane;
-        float y[32], vv[32];
-        const uint4* vrow = reinterpret_cast<const uint4*>(stg + S_V + j * 64);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 raw = vrow[q];
-          const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const float2 f = __bfloat1622float2(hh[x]);
-            vv[8 * q + 2 * x] = f.x;
-            vv[8 * q + 2 * x + 1] = f.y;
-          }
-        }
-        const float eg = gates[j];
-        tmem_ld32(tb + tlane + TM_OY + 32 * ob, y);
-        tmem_wait_ld();
-#pragma unroll
-        for (int v = 0; v < kDVS; ++v)
-          *reinterpret_cast<float*>(tRT + swz_off(v, j, kDVS)) = to_tf32(fmaf(-eg, y[v], vv[v]));
-      }
-      fence_smem_to_async();
-      fence_before_sync();
-      named_bar(1, 128);
-      // ---- U = T R (tf32) ----------------------------------------------------------------------
-      if (warp == 0) {
-        fence_after_sync();
-        const uint64_t dT = sdesc(a + S_PT + WS_T, 16, 1024);
-        const uint32_t id = idesc_tf32(64, 32, false, false);
-#pragma unroll
-        for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32_w(tb + TM_U, kstep(dT, 64, ks), kstep(dRT, kDVS, ks), id, ks > 0);
-        mma_commit_w(mma_bar);
-      }
-      if ((aborted = wait_mma())) break;
-      // ---- U (tf32 [v][j]) and U' = Diag(e^{G_last-G}) U (bf16 hi+lo [v][j]) ------------------
-      {
-        float u[32];
-        tmem_ld32(tb + tlane + TM_U, u);
-        tmem_wait_ld();
-        if (lane < 16) {
-          const int j = 16 * q4 + lane;
-          const float el = gates[64 + j];
-#pragma unroll
-          for (int v = 0; v < kDVS; ++v) {
-            *reinterpret_cast<float*>(tUT + swz_off(v, j, kDVS)) = to_tf32(u[v]);
-            __nv_bfloat16 hi, lo;
-            split_bf16(u[v] * el, hi, lo);
-            const uint32_t off = swz_off_bf16(v, j, kDVS);
-            *reinterpret_cast<__nv_bfloat16*>(tUPH + off) = hi;
-            *reinterpret_cast<__nv_bfloat16*>(tUPL + off) = lo;
-          }
-        }
-      }
-      fence_smem_to_async();
-      fence_before_sync();
-      named_bar(1, 128);
-      // ---- O2 = P U (tf32);  S^T += K^T (U'_hi + U'_lo) (bf16) ----------------------------------
-      if (warp == 0) {
-        // the state update first: the chain continues as soon as it completes, while
-        // P U (needed only for the outputs) runs behind it; the stage is released and
-        // the outputs handed to the loader when both have completed
-        fence_after_sync();
-        const uint64_t dP = sdesc(a + S_PT, 16, 1024);
-        const uint64_t dKT = sdesc(a + S_KT, 16, 1024);
-        const uint32_t ib = idesc_bf16(128, 32);
-#pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks)
-          mma_bf16_w(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPH, kDVS, ks), ib, true);
-#pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks)
-          mma_bf16_w(tb + TM_S, kstep(dKT, 128, ks), kstep(dUPL, kDVS, ks), ib, true);
-        mma_commit_w(mma_bar);
-        const uint32_t it = idesc_tf32(64, 32, false, false);
-#pragma unroll
-        for (int ks = 0; ks < kC / 8; ++ks)
-          mma_tf32_w(tb + TM_O2 + 32 * ob, kstep(dP, 64, ks), kstep(dUT, kDVS, ks), it, ks > 0);
-        mma_commit_w(reinterpret_cast<uint64_t*>(&cs.empty[s]));
-        mma_commit_w(reinterpret_cast<uint64_t*>(&cs.out_full[ob]));
-      }
-      if ((aborted = wait_mma())) break;
-      // ---- new state: the chain's only remaining step before chunk c+1 ----------------------
-      tmem_ld32(tb + tlane + TM_S, st);
-      tmem_wait_ld();
-      write_state_operand();
-      fence_smem_to_async();
-      fence_before_sync();
-      named_bar(1, 128);
-    }
-    if (!aborted && s_final) {
-#pragma unroll
-      for (int vv = 0; vv < kDVS; ++vv) s_final[sbase + (long)(v0 + vv) * kDK + tid] = st[vv];
-    }
-  }
-  fence_before_sync();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, C_TM_COLS);
 }
 
 uint32_t split_spin_limit() {
@@ -766,14 +392,12 @@ uint32_t split_spin_limit() {
   return (uint32_t)strtoul(e, nullptr, 10);
 }
 
-template <typename Tout>
 cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk;
   if (!encode_bthd_bf16(&mq, a.q, TB, a.T, a.H, kDK, 64, kC, true) ||
-      !encode_bthd_bf16(&mk, a.k, TB, a.T, a.H, kDK, 64, kC, true) ||
-      !encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, kDVS, kC, false))
+      !encode_bthd_bf16(&mk, a.k, TB, a.T, a.H, kDK, 64, kC, true))
     return cudaErrorInvalidValue;
   const uint32_t lim = split_spin_limit();
   cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel,
@@ -785,13 +409,7 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   timing_mark(stream, 0);
-  auto carry = gdn_chunk_carry_kernel<Tout>;
-  e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, C_SMEM);
-  if (e != cudaSuccess) return e;
-  carry<<<m.nseq * a.H * (a.dv / kDVS), C_THREADS, C_SMEM, stream>>>(
-      mq, mk, mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H,
-      a.dv, (unsigned int*)a.workspace, lim);
-  e = cudaGetLastError();
+  e = launch_chunk_carry(a, m, lim, stream);
   if (e == cudaSuccess) timing_mark(stream, 1);
   return e;
 }
@@ -800,14 +418,13 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
 
 size_t split_prefill_workspace(int B, int T, int H) {
   const size_t nchunks = ((size_t)T + kC - 1) / kC;
-  return (size_t)B * H * nchunks * kChunkWs;
+  return (size_t)B * H * nchunks * img::kChunkWs;
 }
 
-size_t split_chunk_image_bytes() { return kChunkWs; }
+size_t split_chunk_image_bytes() { return img::kChunkWs; }
 
 cudaError_t launch_prefill_split(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
-  if (a.out_dtype == GDR_F32) return launch_split_t<float>(a, m, stream);
-  return launch_split_t<__nv_bfloat16>(a, m, stream);
+  return launch_split_t(a, m, stream);
 }
 
 }  // namespace gdr
