@@ -624,8 +624,8 @@ bool tc_prefill_supported(const PrefillArgs& a) {
 cudaError_t launch_prefill_kda_tc(const PrefillArgs& a, cudaStream_t stream);  // prefill_kda_tc.cu
 
 // The two-kernel paths (per-chunk prep over the whole GPU, then the carry) need a
-// workspace of 33 KB (GDN) or 128.5 KB (KDA) per chunk; with a smaller workspace the
-// single-kernel kernels run.
+// workspace of 128.5 KB per chunk; with a smaller workspace the single-kernel kernels
+// run.
 size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
   PrefillArgs a{};
   a.in_dtype = GDR_BF16;
