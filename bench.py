@@ -228,7 +228,7 @@ class PrefillRunner:
         # the tensor-core path with a full-size workspace runs a per-chunk prep kernel,
         # then the state carry; the others run one kernel per call
         if self.path == "tensor-core":
-            self.kernels = [f"{w.mixer}_chunk_prep_kernel", f"{w.mixer}_chunk_carry_kernel"]
+            self.kernels = [f"{w.mixer}_chunk_prep_kernel", "state carry (sliced_carry_kernel or row_carry_kernel)"]
             self.kernel_key = f"prefill_two-kernel:{w.name}"
         else:
             self.kernels = ["prefill_simt_kernel"]
@@ -310,7 +310,7 @@ class VarlenRunner:
                                                         int(w.mixer == "kda"))
         self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
         self.kernels = ["varlen index + " + f"{w.mixer}_chunk_prep_kernel",
-                        f"{w.mixer}_chunk_carry_kernel"]
+                        "state carry (sliced_carry_kernel or row_carry_kernel)"]
         self.launches_per_step = 3
         self.kernel_key = f"prefill_two-kernel:{w.name}"
         self.path = "tensor-core"

@@ -1,4 +1,8 @@
-// The state carry shared by the GDN and KDA two-kernel prefills (sm_100a, tcgen05).
+// The value-sliced state carry of the GDN and KDA two-kernel prefills (sm_100a, tcgen05):
+// one CTA per (sequence, head, slice of NV value columns), so one head's carry runs on
+// several SMs at once.  It is taken when there are too few (sequence, head) chains to
+// fill the GPU; otherwise the per-head carry (carry_rows.cu) reads each chunk's operands
+// once instead of once per slice.
 //
 // "Super Apriel: One Checkpoint, Many Speeds", §2A names the two mixers (delta rule with
 // a scalar gate, GDN, and with a per-channel gate, KDA).  Once the prep kernel of either
@@ -9,13 +13,14 @@
 //   O = O1 + P U
 //   S^T <- Diag(e^{G_last}) S0^T + K^ U
 //
-// with Q~ = Q (.) e^G, K~ = K (.) e^G, K^ = (K (.) e^{G_last - G})^T.  One CTA walks the
-// chunks of one (sequence, head, slice of NV value columns) in order.  Its loader
-// warpgroup only copies: each operand group has its own full / empty barrier pair and is
-// refilled for the next chunk as soon as the products that read it have completed; the
-// loader also forms the outputs of the previous chunk.  The carry warpgroup keeps the
-// state as an fp32 TMEM accumulator and a tf32 operand tile.  NV = 64 (two value slices
-// sharing each chunk's operands) is taken when that still gives every SM a chain.
+// with Q~ = Q (.) e^G, K~ = K (.) e^G, K^ = (K (.) e^{G_last - G})^T, each product with the
+// chunk image tile as the A operand (M = 128 token or channel rows) and the value slice
+// as N.  The loader warpgroup only copies: each operand group has its own full / empty
+// barrier pair and is refilled for the next chunk as soon as the products that read it
+// have completed; the loader also forms the outputs of the previous chunk.  The carry
+// warpgroup keeps the state as an fp32 TMEM accumulator and a tf32 operand tile.  NV = 64
+// (two value slices sharing each chunk's operands) is taken when that still gives every
+// SM a chain.
 //
 // Precision: kind::tf32 products with operands rounded to nearest.  Waits are bounded; a
 // give-up records GDR_ERR_TIMEOUT in the workspace status word, drains what was issued,
@@ -84,7 +89,7 @@ struct CarrySmall {
 
 template <int NV, typename Tout>
 __global__ void __launch_bounds__(C_THREADS, 1)
-chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
+sliced_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
                        const unsigned char* __restrict__ ws, const float* __restrict__ s0,
                        Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m,
                        int H, int dv, unsigned int* __restrict__ status, uint32_t spin_limit) {
@@ -388,7 +393,7 @@ chunk_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
 }  // namespace
 
 template <typename Tout>
-cudaError_t launch_carry_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim,
+cudaError_t launch_sliced_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim,
                            cudaStream_t stream) {
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
@@ -405,7 +410,7 @@ cudaError_t launch_carry_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   if (a.dv % 64 == 0 && ctas64 >= sms) {
-    auto carry = chunk_carry_kernel<64, Tout>;
+    auto carry = sliced_carry_kernel<64, Tout>;
     e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CarryLayout<64>::SMEM);
     if (e != cudaSuccess) return e;
@@ -413,7 +418,7 @@ cudaError_t launch_carry_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim
         mv, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H, a.dv,
         (unsigned int*)a.workspace, lim);
   } else {
-    auto carry = chunk_carry_kernel<32, Tout>;
+    auto carry = sliced_carry_kernel<32, Tout>;
     e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CarryLayout<32>::SMEM);
     if (e != cudaSuccess) return e;
@@ -424,12 +429,11 @@ cudaError_t launch_carry_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim
   return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
-                               cudaStream_t stream) {
-  if (a.out_dtype == GDR_F32) return launch_carry_t<float>(a, m, spin_limit, stream);
-  return launch_carry_t<__nv_bfloat16>(a, m, spin_limit, stream);
+cudaError_t launch_carry_sliced(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
+                                cudaStream_t stream) {
+  if (a.out_dtype == GDR_F32) return launch_sliced_t<float>(a, m, spin_limit, stream);
+  return launch_sliced_t<__nv_bfloat16>(a, m, spin_limit, stream);
 }
 
-size_t chunk_image_bytes() { return kChunkWs; }
 
 }  // namespace gdr

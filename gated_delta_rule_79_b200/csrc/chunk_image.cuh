@@ -1,5 +1,5 @@
 // The per-chunk operand images that both two-kernel prefills (GDN and KDA) leave in the
-// workspace for the state carry (carry.cu), and small helpers for the 128-byte-swizzled
+// workspace for the state carry (carry_rows.cu, carry_sliced.cu), and small helpers for the 128-byte-swizzled
 // tf32 tiles they are stored as.  For chunk c of a sequence, with G the chunk-local
 // cumulative log gate (per token for GDN, per token and key channel for KDA):
 //   group A: [Q (.) e^G; K (.) e^G] (128 x 128) and e^{G_last} per key channel

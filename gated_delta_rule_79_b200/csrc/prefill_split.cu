@@ -17,7 +17,7 @@
 // gives T.  It leaves the chunk's operand images for the carry in the workspace
 // (chunk_image.cuh): [Q (.) e^G; K (.) e^G], e^{G_last}, T, (K (.) e^{G_last - G})^T and
 // P as tf32 tiles.  The state carry that walks the chunks in order is shared with KDA
-// (carry.cu).
+// (carry_rows.cu, carry_sliced.cu).
 //
 // Precision: the Gram is exact (bf16 inputs, fp32 accumulation); the carry's products
 // run as kind::tf32 with operands rounded to nearest.  Waits are bounded; a give-up

@@ -34,12 +34,13 @@ __device__ __forceinline__ uint32_t swz_off4(int r, int q, int rows) {
   return (uint32_t)(panel * rows * 128 + r * 128 + (((q & 7) ^ (r & 7)) << 4));
 }
 
-// fp32 -> tf32 with round-to-nearest (the tensor core would otherwise drop the
-// low mantissa bits).
+// fp32 -> tf32, round to nearest with ties away from zero (the tensor core would
+// otherwise drop the low mantissa bits).  Done on the bit pattern: adding half a tf32
+// unit (bit 12) to the sign-magnitude encoding carries into the kept bits exactly when
+// the 13 dropped bits are at least half a unit, which is the rounding cvt.rna.tf32.f32
+// performs, in two integer operations.  Finite inputs only.
 __device__ __forceinline__ float to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
 }
 
 // ---- descriptors -----------------------------------------------------------------------

@@ -15,9 +15,11 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
-@pytest.mark.parametrize("path", ["single-kernel", "two-kernel"])
-def test_bounded_wait_reports_timeout_and_recovers(mixer, path):
+@pytest.mark.parametrize("path", ["single-kernel", "two-kernel rows", "two-kernel sliced"])
+def test_bounded_wait_reports_timeout_and_recovers(mixer, path, monkeypatch):
     import gated_delta_rule_79_b200 as g
+    if path.startswith("two-kernel"):
+        monkeypatch.setenv("GDR_CARRY", path.split()[1])
     kda = mixer == "kda"
     w = Workload("fi", mixer, 1, 2, 100, 128, 128, "bf16", "randn")
     x = {k: v.cuda() for k, v in make_inputs(w, seed=11).items()}

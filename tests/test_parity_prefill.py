@@ -200,11 +200,58 @@ def test_in_place_state_carry(mixer):
 
 
 @pytest.mark.parametrize("dv", [128, 64])
-def test_kda_carry_with_64_value_columns(dv):
-    """With enough (sequence, head) chains the KDA carry takes 64 value columns per CTA
-    (two slices sharing each chunk's operands): 3 x 50 heads run that way."""
+def test_kda_carry_with_64_value_columns(dv, monkeypatch):
+    """With enough (sequence, head) chains the value-sliced carry takes 64 value columns
+    per CTA (two slices sharing each chunk's operands): 3 x 50 heads run that way."""
+    monkeypatch.setenv("GDR_CARRY", "sliced")
     w = Workload("wide", "kda", 3, 50, 130, 128, dv, "bf16", "randn")
     x = make_inputs(w, seed=77)
     o, s = gpu_prefill("kda", x, out_dtype=torch.float32)
     o_ref, s_ref = ref_prefill(x)
     check(o, s, o_ref, s_ref, TOL["bf16"], f"kda 64-column carry dv={dv}")
+
+
+@pytest.mark.parametrize("carry", ["rows", "sliced"])
+@pytest.mark.parametrize("mixer", ["gdn", "kda"])
+@pytest.mark.parametrize("dv", [128, 64, 32])
+@pytest.mark.parametrize("gates", ["slow", "zero_some"])
+def test_both_carries(carry, mixer, dv, gates, monkeypatch):
+    """Either state carry, forced (the per-head one runs all value rows of a head in one
+    CTA, the value-sliced one spreads them): a ragged tail, an entering state, gates
+    that make the carry matter."""
+    monkeypatch.setenv("GDR_CARRY", carry)
+    w = Workload("carry", mixer, 2, 3, 200, 128, dv, "bf16", "randn")
+    x = make_inputs(w, seed=dv + 11, gates=gates)
+    o, s = gpu_prefill(mixer, x, out_dtype=torch.float32)
+    o_ref, s_ref = ref_prefill(x)
+    check(o, s, o_ref, s_ref, TOL["bf16"], f"{carry} carry {mixer} dv={dv} gates={gates}")
+
+
+@pytest.mark.parametrize("carry", ["rows", "sliced"])
+@pytest.mark.parametrize("mixer", ["gdn", "kda"])
+def test_both_carries_bf16_out_in_place(carry, mixer, monkeypatch):
+    """bf16 outputs and the final state written over the entering one."""
+    import gated_delta_rule_79_b200 as g
+    monkeypatch.setenv("GDR_CARRY", carry)
+    w = Workload("carry16", mixer, 3, 2, 129, 128, 128, "bf16", "randn")
+    x = make_inputs(w, seed=21, gates="slow")
+    o_ref, s_ref = ref_prefill(x)
+    t = {k: v.cuda() for k, v in x.items()}
+    fn = g.kda_prefill if mixer == "kda" else g.gdn_prefill
+    state = t["s0"].clone()
+    o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{carry} carry bf16 in place")
+
+
+def test_many_chains_take_the_per_head_carry():
+    """40 sequences x 4 heads x 4 value slices exceed the SM count, so the automatic
+    choice is the per-head carry; checked against the oracle on sampled chains."""
+    w = Workload("many", "gdn", 40, 4, 96, 128, 128, "bf16", "randn")
+    x = make_inputs(w, seed=31, gates="slow")
+    o, s = gpu_prefill("gdn", x, out_dtype=torch.float32)
+    picks = [0, 17, 39]
+    sub = {k: (v[picks] if v is not None else None) for k, v in x.items()}
+    o_ref, s_ref = ref_prefill(sub)
+    check(o[picks], s[picks], o_ref, s_ref, TOL["bf16"], "many chains")

@@ -41,11 +41,13 @@ def _run(mixer, x, cu, pool, slots, out_dtype=None):
     return o
 
 
+@pytest.mark.parametrize("carry", ["rows", "sliced"])
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
 @pytest.mark.parametrize("dv", [128, 32])
-def test_varlen_ragged(mixer, dv):
+def test_varlen_ragged(mixer, dv, carry, monkeypatch):
     """Lengths across the chunk edges (and an empty sequence), permuted slots in a pool
-    with unused slots; outputs in fp32 and every slot checked."""
+    with unused slots; outputs in fp32 and every slot checked, through either carry."""
+    monkeypatch.setenv("GDR_CARRY", carry)
     lens = [70, 0, 1, 64, 129, 13, 200, 63]
     H = 3
     x, cu = _packed(mixer, lens, H, dv, seed=5)
