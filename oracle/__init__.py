@@ -24,7 +24,10 @@ recurrent   the definition, token by token (the oracle proper); decode_step and
             prefill_varlen runs packed sequences from a pool of state slots
 chunked     an independent fp64 chunk-wise restatement, used only to pin the
             chunk algebra against the definition
+backward    the gradients of the recurrence (inputs, gates and initial state),
+            token by token in reverse
 """
 
 from .recurrent import gated_delta_rule, decode_step, verify_steps, prefill_varlen  # noqa: F401
 from .chunked import chunked_gated_delta_rule  # noqa: F401
+from .backward import gated_delta_rule_backward  # noqa: F401
