@@ -8,8 +8,15 @@ Workloads (synthetic inputs, recipe in synth/):
   decode_gdn   256 sequences x 32 heads, d=128, 512 one-token steps, GDN gates
   decode_kda   same with KDA gates
   kda_long     KDA prefill with a carried state, B=4 H=32 T=65536 d=128
+  verify_gdn   multi-token verify (K=4) for 256 sequences x 32 heads, GDN / KDA gates
+  verify_kda
+  gdn_varlen   64 prompts packed with per-sequence state slots, GDN / KDA gates
+  kda_varlen
+  gdn_backward the gradients of the gdn_prefill / kda_prefill shapes (fp32 arithmetic)
+  kda_backward
 
-One step is one pass of the workload: one prefill call, or 512 decode calls.
+One step is one pass of the workload: one prefill (or verify, packed prefill,
+gradient) call, or 512 decode calls.
 `value` is whole-job tokens/s (a token = one position of one sequence, all H
 heads) with inputs resident in HBM; `e2e` is the same through the public API
 with pinned host buffers copied in and results copied out inside the timed
@@ -33,7 +40,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, device_inputs, slice_inputs, tokens, varlen_lengths  # noqa: E402
+from synth import (WORKLOADS, device_inputs, slice_inputs, slice_seed, tokens,  # noqa: E402
+                   varlen_lengths)
 
 METRIC = "GDN/KDA prefill tokens/s and decode tokens/s at 1 B200; % of roofline"
 L2_BYTES = 126 * 2 ** 20
@@ -62,6 +70,12 @@ def algorithmic(w):
         per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
         return (1 + w.T) * state + th * per_th, th * 6 * w.dk * w.dv
     a_bytes = 4 * (w.dk if w.mixer == "kda" else 1)
+    if w.backward:
+        # inputs q, k, v, alpha, beta and dL/do read once; dq, dk, dv, dalpha, dbeta
+        # written once (fp32); dL/dS_T read and ds0 written.  Flops of the token-level
+        # reverse: the forward recurrence (5 d_k d_v) plus the reverse step (16 d_k d_v).
+        per_th = esz * (2 * w.dk + 2 * w.dv) + a_bytes + 4 + 4 * (2 * w.dk + w.dv) + a_bytes + 4
+        return th * per_th + 2 * state, th * 21 * w.dk * w.dv
     per_th = esz * (2 * w.dk + w.dv) + a_bytes + 4 + esz * w.dv
     # the final states are written; initial states read when the workload has them
     nbytes = th * per_th + state + (state if w.state == "randn" else 0)
@@ -70,12 +84,21 @@ def algorithmic(w):
     return nbytes, flops
 
 
+def alu_peak_tflops(peaks):
+    """fp32 CUDA-core peak of a B200 from its unit counts and clock: 148 SMs x 128 fp32
+    lanes x 2 flops per fused multiply-add x the maximum SM clock."""
+    mhz = peaks.get("sm_max_mhz") or 1965.0
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        out = {k: float(d[k]) for k in FALLBACK_PEAKS}
+        out["sm_max_mhz"] = float(d.get("sm_max_mhz", 1965.0))
+        return out, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
 
@@ -324,6 +347,38 @@ class VarlenRunner:
                 workspace=self.ws)
 
 
+class BackwardRunner:
+    """One gradient call per step (dq, dk, dv, dalpha, dbeta, ds0 of the whole
+    workload); two rotating input sets (each above L2)."""
+
+    def __init__(self, w, dev, seed):
+        import gated_delta_rule_79_b200 as g
+        self.g, self.w, self.dev = g, w, dev
+        self.fn = g.kda_backward if w.mixer == "kda" else g.gdn_backward
+        self.sets = []
+        for i in range(2):
+            x = device_inputs(w, dev, seed=seed + i)
+            gen = torch.Generator(device=dev).manual_seed(seed + 50 + i)
+            x["do"] = torch.randn((w.B, w.T, w.H, w.dv), generator=gen, device=dev).to(
+                w.torch_dtype)
+            x["dsf"] = torch.randn((w.B, w.H, w.dv, w.dk), generator=gen, device=dev)
+            self.sets.append(x)
+        need = g.backward_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda")
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.kernels = ["gdr_backward_kernel"]
+        self.kernel_key = f"backward:{w.name}"
+        self.launches_per_step = 1
+        self.path = "backward (CUDA cores, fp32)"
+        set_bytes = sum(t.numel() * t.element_size() for t in self.sets[0].values()
+                        if t is not None)
+        self.l2_note = f"2 rotating input sets of {set_bytes / 2**20:.0f} MiB (> L2)"
+
+    def step(self, i):
+        x = self.sets[i % 2]
+        self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"], x["do"], x["dsf"],
+                workspace=self.ws)
+
+
 def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
     """Warm up, then time exactly `steps` steps with CUDA events on the launching
     stream, bracketed by a barrier and a synchronize on both sides.  Also records
@@ -348,7 +403,7 @@ def time_device(runner, steps, warmup, dev, active, soak_s=0.5):
           for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    per_kernel = not (runner.w.decode or runner.w.verify)
+    per_kernel = not (runner.w.decode or runner.w.verify or runner.w.backward)
     if per_kernel:
         runner.g.timing_start()
     t0.record(stream)
@@ -411,6 +466,31 @@ def time_e2e(w, dev, steps, warmup, seed):
             fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], cu, pool, o=o,
                workspace=ws)
             o_host.copy_(o, non_blocking=True)
+    elif w.backward:
+        fn = g.kda_backward if w.mixer == "kda" else g.gdn_backward
+        keys = ("q", "k", "v", "alpha", "beta")
+        gen = torch.Generator(device=dev).manual_seed(seed + 150)
+        x["do"] = torch.randn((w.B, w.T, w.H, w.dv), generator=gen, device=dev).to(w.torch_dtype)
+        x["dsf"] = torch.randn((w.B, w.H, w.dv, w.dk), generator=gen, device=dev)
+        keys = keys + ("do", "dsf")
+        host = {k: x[k].cpu().pin_memory() for k in keys}
+        dbuf = {k: torch.empty_like(x[k]) for k in keys}
+        need = g.backward_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda")
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        out_host = None
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        shapes = [(w.B, w.T, w.H, w.dk), (w.B, w.T, w.H, w.dk), (w.B, w.T, w.H, w.dv),
+                  tuple(x["alpha"].shape), (w.B, w.T, w.H), (w.B, w.H, w.dv, w.dk)]
+        out_host = [torch.empty(sh, dtype=torch.float32).pin_memory() for sh in shapes]
+        d2h = sum(t.numel() * 4 for t in out_host)
+
+        def step():
+            for key in keys:
+                dbuf[key].copy_(host[key], non_blocking=True)
+            grads = fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], None,
+                       dbuf["do"], dbuf["dsf"], workspace=ws)
+            for hbuf, gr in zip(out_host, grads):
+                hbuf.copy_(gr, non_blocking=True)
     elif w.verify:
         fn = g.kda_verify if w.mixer == "kda" else g.gdn_verify
         keys = ("q", "k", "v", "alpha", "beta")
@@ -482,6 +562,15 @@ def _oracle_slice(args):
     x = slice_inputs(w.with_(T=t_sample), b, h)
     col = lambda key: x[key][None, :, None].double().numpy()  # noqa: E731
     s0 = None if x["s0"] is None else x["s0"][None, None].double().numpy()
+    if w.backward:
+        from oracle import gated_delta_rule_backward
+        g = torch.Generator().manual_seed(slice_seed(7, b, h))
+        do = torch.randn((1, t_sample, 1, w.dv), generator=g).double().numpy()
+        dsf = torch.randn((1, 1, w.dv, w.dk), generator=g).double().numpy()
+        t = time.perf_counter()
+        gated_delta_rule_backward(col("q"), col("k"), col("v"), col("alpha"), col("beta"), s0,
+                                  do, dsf)
+        return time.perf_counter() - t
     t = time.perf_counter()
     if w.decode:
         st = s0
@@ -513,6 +602,9 @@ class OracleTimer:
             t_cal = min(w.T, 64)
             per_token_head = _oracle_slice((w.name, 0, 0, t_cal)) / t_cal
             self.t_sample = max(1, min(w.T, int(budget_s / max(per_token_head, 1e-9))))
+            if w.backward:
+                # the backward oracle keeps every state of its sample in memory
+                self.t_sample = min(self.t_sample, 512)
             self.tokens_per_unit = 1
             what = f"{self.t_sample} tokens"
         self.chains = [(w.name, i // w.H, i % w.H, self.t_sample) for i in range(self.cores)]
@@ -582,7 +674,8 @@ def main():
     active = dist_init(world, "nccl")
     peaks, peak_kind = load_peaks()
     runner = (DecodeRunner if w.decode else VerifyRunner if w.verify
-              else VarlenRunner if w.varlen else PrefillRunner)(w, dev, seed=1000 * rank)
+              else VarlenRunner if w.varlen else BackwardRunner if w.backward
+              else PrefillRunner)(w, dev, seed=1000 * rank)
     clocks = ClockSampler(dev.index)
     clocks.start()
     total_ms, per, kernel_ms = time_device(runner, steps, warmup, dev, active)
@@ -617,8 +710,19 @@ def main():
                                for n, m in zip(runner.kernels, kernel_ms)]
         dom = max(range(len(kernel_ms)), key=lambda i: kernel_ms[i])
         roofline["dominant"] = runner.kernels[dom] if dom < len(runner.kernels) else None
+    if w.backward:
+        # fp32 arithmetic on the CUDA cores bounds the gradient pass (its HBM time is a
+        # tenth of the fp32 time), so the roofline is the fp32 CUDA-core peak
+        alu = alu_peak_tflops(peaks)
+        roofline = {"bound": "alu", "achieved": tflops, "peak": alu, "unit": "TFLOP/s",
+                    "frac": tflops / alu, "traffic": traffic,
+                    "peak_source": "unit counts: 148 SMs x 128 fp32 lanes x 2 x max SM clock",
+                    "algorithmic_flops_per_launch": flops_launch, "launch_ms": launch_ms,
+                    "hbm": {"achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": hbm / peaks["hbm_gbs"],
+                            "algorithmic_bytes_per_launch": bytes_launch}}
     extra = {}
-    if not (w.decode or w.verify):
+    if not (w.decode or w.verify or w.backward):
         extra["roofline_tensor"] = {
             "bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
@@ -630,7 +734,8 @@ def main():
             "dtype": "bf16" if runner.path == "tensor-core" else "f32",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                       "tokens_per_step": ntok, "in_dtype": w.dtype, "out_dtype": "bf16",
+                       "tokens_per_step": ntok, "in_dtype": w.dtype,
+                       "out_dtype": "f32" if w.backward else "bf16",
                        "chunk": 64,
                        "kernel": runner.path, "l2": runner.l2_note,
                        "clocks_window": "0.5 s soak of the same steps, then the timed region",

@@ -24,7 +24,8 @@ EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
            "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop",
            "gdn_verify", "kda_verify", "gdr_prefill_varlen_workspace_bytes",
-           "gdn_prefill_varlen", "kda_prefill_varlen"]
+           "gdn_prefill_varlen", "kda_prefill_varlen", "gdr_backward_workspace_bytes",
+           "gdn_backward", "kda_backward"]
 
 
 class GdrError(RuntimeError):
@@ -64,6 +65,13 @@ def _load():
         f = getattr(lib, name)
         f.restype = i
         f.argtypes = [vp, vp, vp, fp, fp, vp, vp, fp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.gdr_backward_workspace_bytes.restype = sz
+    lib.gdr_backward_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    for name in ("gdn_backward", "kda_backward"):
+        f = getattr(lib, name)
+        f.restype = i
+        f.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp,
+                      i, i, i, i, i, i, i, vp, sz, vp]
     lib.gdn_prefill_noalloc.restype = i
     lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdr_prefill_path.restype = i
@@ -339,6 +347,59 @@ def kda_verify(q, k, v, alpha, beta, state, *, snapshots=True, out_dtype=None, o
                stream=None):
     """Kimi Delta Attention (alpha [N, K, H, d_k]); as ``gdn_verify``."""
     return _verify(True, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream)
+
+
+def _backward(kda, q, k, v, alpha, beta, s0, do, ds_final, workspace, stream):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, d_k]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors (there is no CPU path)")
+    dt = q.dtype
+    _need(q, "q", (B, T, H, dk), dt, dev)
+    _need(k, "k", (B, T, H, dk), dt, dev)
+    _need(v, "v", (B, T, H, dv), dt, dev)
+    _need(alpha, "alpha", (B, T, H, dk) if kda else (B, T, H), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if s0 is not None:
+        _need(s0, "s0", (B, H, dv, dk), torch.float32, dev)
+    _need(do, "do", (B, T, H, dv), None, dev)
+    if ds_final is not None:
+        _need(ds_final, "ds_final", (B, H, dv, dk), torch.float32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq = torch.empty((B, T, H, dk), **f32)
+    dk_ = torch.empty((B, T, H, dk), **f32)
+    dv_ = torch.empty((B, T, H, dv), **f32)
+    dalpha = torch.empty(alpha.shape, **f32)
+    dbeta = torch.empty((B, T, H), **f32)
+    ds0 = torch.empty((B, H, dv, dk), **f32)
+    need = lib.gdr_backward_workspace_bytes(B, T, H, dk, dv, int(kda))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    nws = workspace.numel() * workspace.element_size()
+    fn = lib.kda_backward if kda else lib.gdn_backward
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(s0), _ptr(do),
+              _ptr(ds_final), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dalpha), _ptr(dbeta),
+              _ptr(ds0), B, T, H, dk, dv, _code(dt), _code(do.dtype), _ptr(workspace), nws,
+              _stream(dev, stream)))
+    return dq, dk_, dv_, dalpha, dbeta, ds0
+
+
+def gdn_backward(q, k, v, alpha, beta, s0, do, ds_final=None, *, workspace=None, stream=None):
+    """Gradients (dq, dk, dv, dalpha [B,T,H], dbeta, ds0), all fp32, of
+    L = sum <do, o> + <ds_final, S_T> for gdn_prefill(q, k, v, alpha, beta, s0)."""
+    return _backward(False, q, k, v, alpha, beta, s0, do, ds_final, workspace, stream)
+
+
+def kda_backward(q, k, v, alpha, beta, s0, do, ds_final=None, *, workspace=None, stream=None):
+    """As gdn_backward with the per-channel gate: dalpha is [B, T, H, d_k]."""
+    return _backward(True, q, k, v, alpha, beta, s0, do, ds_final, workspace, stream)
+
+
+def backward_workspace_bytes(B, T, H, dk, dv, kda):
+    return lib.gdr_backward_workspace_bytes(B, T, H, dk, dv, int(kda))
 
 
 def prefill_path(dk, dv, dtype, kda):

@@ -153,6 +153,46 @@ static gdr_status verify(bool kda, const void* q, const void* k, const void* v,
   return ok();
 }
 
+static gdr_status backward(bool kda, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, const float* s0,
+                           const void* dO, const float* ds_final, float* dq, float* dkk,
+                           float* dvv, float* dalpha, float* dbeta, float* ds0, int B, int T,
+                           int H, int dk, int dv, int in_dtype, int do_dtype, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  const char* fn = kda ? "kda_backward" : "gdn_backward";
+  if (B < 0 || T < 0 || H < 0)
+    return fail(GDR_ERR_INVALID_ARG, "%s: negative size B=%d T=%d H=%d", fn, B, T, H);
+  if (!head_ok(dk) || !head_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "%s: d_k=%d d_v=%d (supported: 32, 64, 128)", fn, dk, dv);
+  if (!dtype_ok(in_dtype) || !dtype_ok(do_dtype))
+    return fail(GDR_ERR_INVALID_ARG, "%s: bad dtype in=%d do=%d", fn, in_dtype, do_dtype);
+  if ((long long)B * H > (1LL << 24) || T > (1 << 28) ||
+      (long long)B * T * H * (dk > dv ? dk : dv) > (1LL << 40))
+    return fail(GDR_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if (B == 0 || H == 0) return ok();
+  const void* need_ptrs[] = {q, k, v, alpha, beta, dO, dq, dkk, dvv, dalpha, dbeta, ds0};
+  const char* names[] = {"q", "k", "v", "alpha", "beta", "do", "dq", "dk", "dv", "dalpha",
+                         "dbeta", "ds0"};
+  for (int i = 0; i < 12; ++i) {
+    if (!need_ptrs[i] && (T > 0 || i == 11))
+      return fail(GDR_ERR_INVALID_ARG, "%s: %s is NULL", fn, names[i]);
+    if (!aligned16(need_ptrs[i]))
+      return fail(GDR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
+  }
+  if ((s0 && !aligned16(s0)) || (ds_final && !aligned16(ds_final)))
+    return fail(GDR_ERR_INVALID_ARG, "%s: s0/ds_final not 16-byte aligned", fn);
+  const size_t need = backward_workspace_bytes(B, T, H, dk, dv);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+    return fail(GDR_ERR_INVALID_ARG,
+                "%s: workspace of %zu bytes needed (gdr_backward_workspace_bytes), 16-byte "
+                "aligned", fn, need);
+  BackwardArgs a{q, k, v, alpha, beta, s0, dO, ds_final, dq, dkk, dvv, dalpha, dbeta, ds0,
+                 B, T, H, dk, dv, in_dtype, do_dtype, kda, workspace};
+  cudaError_t e = launch_backward(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return ok();
+}
+
 }  // namespace gdr
 
 extern "C" {
@@ -209,6 +249,35 @@ gdr_status kda_verify(const void* q, const void* k, const void* v, const float* 
                       int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
   return gdr::verify(true, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
                      out_dtype, stream);
+}
+
+size_t gdr_backward_workspace_bytes(int B, int T, int H, int dk, int dv, int kda) {
+  (void)kda;
+  if (B < 0 || T < 0 || H < 0 || !gdr::head_ok(dk) || !gdr::head_ok(dv)) return 0;
+  if ((long long)B * H > (1LL << 24) || T > (1 << 28)) return 0;
+  return gdr::backward_workspace_bytes(B, T, H, dk, dv);
+}
+
+gdr_status gdn_backward(const void* q, const void* k, const void* v, const float* alpha,
+                        const float* beta, const float* s0, const void* dO,
+                        const float* ds_final, float* dq, float* dk_, float* dv_,
+                        float* dalpha, float* dbeta, float* ds0, int B, int T, int H, int dk,
+                        int dv, int in_dtype, int do_dtype, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return gdr::backward(false, q, k, v, alpha, beta, s0, dO, ds_final, dq, dk_, dv_, dalpha,
+                       dbeta, ds0, B, T, H, dk, dv, in_dtype, do_dtype, workspace, ws_bytes,
+                       stream);
+}
+
+gdr_status kda_backward(const void* q, const void* k, const void* v, const float* alpha,
+                        const float* beta, const float* s0, const void* dO,
+                        const float* ds_final, float* dq, float* dk_, float* dv_,
+                        float* dalpha, float* dbeta, float* ds0, int B, int T, int H, int dk,
+                        int dv, int in_dtype, int do_dtype, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return gdr::backward(true, q, k, v, alpha, beta, s0, dO, ds_final, dq, dk_, dv_, dalpha,
+                       dbeta, ds0, B, T, H, dk, dv, in_dtype, do_dtype, workspace, ws_bytes,
+                       stream);
 }
 
 int gdr_prefill_path(int dk, int dv, int in_dtype, int kda) {

@@ -72,6 +72,30 @@ cudaError_t launch_carry_sliced(const PrefillArgs& a, const ChunkMap& m, uint32_
                                 cudaStream_t stream);
 size_t chunk_image_bytes();
 
+// Gradients of a dense prefill (backward.cu).
+struct BackwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  const float* beta;
+  const float* s0;        // may be null (zeros)
+  const void* dO;
+  const float* ds_final;  // may be null (zeros)
+  float* dq_out;
+  float* dk_out;
+  float* dv_out;
+  float* dalpha;
+  float* dbeta;
+  float* ds0;
+  int B, T, H, dk, dv;
+  int in_dtype, do_dtype;
+  bool kda;
+  void* workspace;
+};
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
+
 // Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
 int report_error(int s, const char* msg);
 

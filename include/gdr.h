@@ -235,6 +235,50 @@ GDR_API gdr_status kda_verify(const void* q, const void* k, const void* v,
                       void* o, int N, int K, int H, int dk, int dv,
                       int in_dtype, int out_dtype, void* stream);
 
+/* Gradients of the mixers.  "Super Apriel: One Checkpoint, Many Speeds", §2B (Training
+ * Recipe): the mixers are trained (stochastic distillation, then supervised fine-tuning),
+ * so the recurrence of §2A is differentiated with respect to its inputs, gates and
+ * initial state.  For a dense batch with the forward arguments of gdn_prefill /
+ * kda_prefill, and the gradients of a loss L with respect to the outputs and the final
+ * state:
+ *
+ *   dO        [B, T, H, d_v]   do_dtype, dL/do
+ *   ds_final  [B, H, d_v, d_k] fp32 dL/dS_T, or NULL for zeros
+ *
+ * writes (all fp32, none may overlap another argument)
+ *
+ *   dq, dk    [B, T, H, d_k]
+ *   dv        [B, T, H, d_v]
+ *   dalpha    GDN: [B, T, H];  KDA: [B, T, H, d_k]   (with respect to alpha itself)
+ *   dbeta     [B, T, H]
+ *   ds0       [B, H, d_v, d_k] (dL/ds0; written also when s0 is NULL)
+ *
+ * d_k, d_v in {32, 64, 128}; in_dtype and do_dtype GDR_F32 or GDR_BF16; any T >= 0
+ * (T == 0 writes ds0 = ds_final).  The gates enter as given: alpha = 0 is exact here
+ * (the forward kernels floor log alpha at -GDR_LOG_GATE_FLOOR).  The workspace must hold
+ * gdr_backward_workspace_bytes(B, T, H, d_k, d_v, kda) bytes, 16-byte aligned (no zero
+ * fill needed): the state entering every chunk of 64 tokens and two fp32 values per
+ * token and value channel.  Pointers are device pointers, 16-byte aligned.  Results are
+ * deterministic (no atomics). */
+GDR_API size_t gdr_backward_workspace_bytes(int B, int T, int H, int dk, int dv, int kda);
+GDR_API gdr_status gdn_backward(const void* q, const void* k, const void* v,
+                        const float* alpha, const float* beta, const float* s0,
+                        const void* dO, const float* ds_final,
+                        float* dq, float* dk_out, float* dv_out, float* dalpha,
+                        float* dbeta, float* ds0,
+                        int B, int T, int H, int dk, int dv,
+                        int in_dtype, int do_dtype,
+                        void* workspace, size_t ws_bytes, void* stream);
+/* Same contract with the per-channel gate alpha [B, T, H, d_k] and dalpha likewise. */
+GDR_API gdr_status kda_backward(const void* q, const void* k, const void* v,
+                        const float* alpha, const float* beta, const float* s0,
+                        const void* dO, const float* ds_final,
+                        float* dq, float* dk_out, float* dv_out, float* dalpha,
+                        float* dbeta, float* ds0,
+                        int B, int T, int H, int dk, int dv,
+                        int in_dtype, int do_dtype,
+                        void* workspace, size_t ws_bytes, void* stream);
+
 /* Which prefill kernel a call with these parameters runs: 1 = the bf16
  * tensor-core (tcgen05) kernel, 0 = the fp32 CUDA-core kernel, -1 = the
  * parameters are not supported.  Pure host query, no CUDA call. */

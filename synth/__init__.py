@@ -16,6 +16,8 @@ Workloads (all inputs synthetic; the pages publish no dataset for the mixer):
   verify_kda    ~ 0.02 N(0,1), bf16 q/k/v; GDN and KDA gates (B = N, T = K)
   gdn_varlen    64 prompts packed along the tokens, H=32, d=128, bf16, each from its
   kda_varlen    own slot of a state pool ~ 0.02 N(0,1); lengths from varlen_lengths
+  gdn_backward  the gradients of the gdn_prefill / kda_prefill shapes; dL/do ~ N(0,1)
+  kda_backward  (bf16) and dL/dS_T ~ N(0,1) (fp32), drawn after the inputs
 
 Recipe per (batch b, head h) slice, one ``torch.Generator`` (CPU) seeded with
 ``slice_seed(seed, b, h)``, drawing in this fixed order:
@@ -56,6 +58,7 @@ class Workload:
     decode: bool = False
     verify: bool = False  # K tokens (the T axis) from a carried state, snapshots kept
     varlen: bool = False  # B sequences of varlen_lengths(w) tokens packed (T: median)
+    backward: bool = False  # the gradients of the prefill of these shapes
 
     @property
     def torch_dtype(self):
@@ -80,6 +83,10 @@ WORKLOADS = {
                            varlen=True),
     "kda_varlen": Workload("kda_varlen", "kda", 64, 32, 256, 128, 128, "bf16", "randn",
                            varlen=True),
+    "gdn_backward": Workload("gdn_backward", "gdn", 1, 32, 4096, 128, 128, "bf16", "zeros",
+                             backward=True),
+    "kda_backward": Workload("kda_backward", "kda", 1, 32, 4096, 128, 128, "bf16", "zeros",
+                             backward=True),
 }
 
 
