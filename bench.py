@@ -14,6 +14,8 @@ Workloads (synthetic inputs, recipe in synth/):
   kda_varlen
   gdn_backward the gradients of the gdn_prefill / kda_prefill shapes (fp32 arithmetic)
   kda_backward
+  gdn_prefill_prologue, kda_prefill_prologue, decode_gdn_prologue: the same calls with
+               the fused prologue (raw q, k normalised and the gates formed in-kernel)
 
 One step is one pass of the workload: one prefill (or verify, packed prefill,
 gradient) call, or 512 decode calls.
@@ -263,7 +265,7 @@ class PrefillRunner:
         x = self.sets[i % len(self.sets)]
         self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"],
                 o=self.o[i % len(self.sets)], s_final=self.s[i % len(self.sets)],
-                workspace=self.ws)
+                workspace=self.ws, prologue=self.w.prologue)
 
 
 class DecodeRunner:
@@ -286,7 +288,7 @@ class DecodeRunner:
         x = self.x
         for t in range(self.w.T):
             self.fn(x["q"][t], x["k"][t], x["v"][t], x["alpha"][t], x["beta"][t], self.state,
-                    o=self.o)
+                    o=self.o, prologue=self.w.prologue)
 
 
 class VerifyRunner:
@@ -440,7 +442,8 @@ def time_e2e(w, dev, steps, warmup, seed):
             for t in range(w.T):
                 for key in dbuf:
                     dbuf[key].copy_(host[key][t], non_blocking=True)
-                fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o)
+                fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o,
+                   prologue=w.prologue)
                 o_host[t].copy_(o, non_blocking=True)
     elif w.varlen:
         fn = g.kda_prefill_varlen if w.mixer == "kda" else g.gdn_prefill_varlen
@@ -523,7 +526,7 @@ def time_e2e(w, dev, steps, warmup, seed):
             for key in dbuf:
                 dbuf[key].copy_(host[key], non_blocking=True)
             fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], dbuf.get("s0"),
-               o=o, s_final=s, workspace=ws)
+               o=o, s_final=s, workspace=ws, prologue=w.prologue)
             o_host.copy_(o, non_blocking=True)
             s_host.copy_(s, non_blocking=True)
     for _ in range(warmup):
@@ -560,6 +563,13 @@ def _oracle_slice(args):
                          x["s0"][None, None].double().numpy())
         return time.perf_counter() - t
     x = slice_inputs(w.with_(T=t_sample), b, h)
+    if w.prologue:
+        from oracle import apply_prologue
+        qk = apply_prologue(x["q"].double().numpy(), x["k"].double().numpy(),
+                            x["alpha"].double().numpy(), l2norm=bool(w.prologue & 1),
+                            gate_logit=bool(w.prologue & 2), bf16=w.dtype == "bf16")
+        x = dict(x, q=torch.from_numpy(qk[0]), k=torch.from_numpy(qk[1]),
+                 alpha=torch.from_numpy(qk[2]))
     col = lambda key: x[key][None, :, None].double().numpy()  # noqa: E731
     s0 = None if x["s0"] is None else x["s0"][None, None].double().numpy()
     if w.backward:
@@ -736,7 +746,7 @@ def main():
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "tokens_per_step": ntok, "in_dtype": w.dtype,
                        "out_dtype": "f32" if w.backward else "bf16",
-                       "chunk": 64,
+                       "chunk": 64, "prologue": w.prologue,
                        "kernel": runner.path, "l2": runner.l2_note,
                        "clocks_window": "0.5 s soak of the same steps, then the timed region",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},

@@ -9,7 +9,7 @@ them without a built ``libgdr.so`` raises ImportError (there is no fallback).
 
 _PUBLIC = ("gdn_prefill", "kda_prefill", "gdn_decode", "kda_decode", "gdn_verify", "kda_verify",
            "gdn_prefill_varlen", "kda_prefill_varlen", "gdn_backward", "kda_backward",
-           "backward_workspace_bytes",
+           "backward_workspace_bytes", "PROLOGUE_L2NORM_QK", "PROLOGUE_GATE_LOGIT",
            "VERIFY_MAX_TOKENS", "prefill_workspace",
            "workspace_status", "prefill_path", "timing_start", "timing_stop", "GdrError", "lib", "LIB_PATH", "EXPORTS", "GDR_OK",
            "GDR_ERR_INVALID_ARG", "GDR_ERR_UNSUPPORTED", "GDR_ERR_CUDA", "GDR_ERR_TIMEOUT",

@@ -25,7 +25,13 @@ EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_
            "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop",
            "gdn_verify", "kda_verify", "gdr_prefill_varlen_workspace_bytes",
            "gdn_prefill_varlen", "kda_prefill_varlen", "gdr_backward_workspace_bytes",
-           "gdn_backward", "kda_backward"]
+           "gdn_backward", "kda_backward", "gdn_prefill_ex", "kda_prefill_ex", "gdn_decode_ex",
+           "kda_decode_ex", "gdn_verify_ex", "kda_verify_ex", "gdn_prefill_varlen_ex",
+           "kda_prefill_varlen_ex"]
+
+# fused prologue flags of the *_ex entry points (prologue= keyword below)
+PROLOGUE_L2NORM_QK = 1   # q, k raw: L2-normalised per (token, head) inside the kernels
+PROLOGUE_GATE_LOGIT = 2  # alpha holds x: the gate is exp(-softplus(x))
 
 
 class GdrError(RuntimeError):
@@ -65,6 +71,11 @@ def _load():
         f = getattr(lib, name)
         f.restype = i
         f.argtypes = [vp, vp, vp, fp, fp, vp, vp, fp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    for name in ("gdn_prefill", "kda_prefill", "gdn_decode", "kda_decode", "gdn_verify",
+                 "kda_verify", "gdn_prefill_varlen", "kda_prefill_varlen"):
+        f = getattr(lib, name + "_ex")
+        f.restype = i
+        f.argtypes = list(getattr(lib, name).argtypes) + [ctypes.c_uint]
     lib.gdr_backward_workspace_bytes.restype = sz
     lib.gdr_backward_workspace_bytes.argtypes = [i, i, i, i, i, i]
     for name in ("gdn_backward", "kda_backward"):
@@ -91,6 +102,13 @@ lib = _load()
 def _check(status):
     if status != GDR_OK:
         raise GdrError(status, lib.gdr_last_error().decode())
+
+
+def _pick(name, prologue):
+    """The plain entry point, or its fused-prologue variant with the flags appended."""
+    if prologue:
+        return getattr(lib, name + "_ex"), (int(prologue),)
+    return getattr(lib, name), ()
 
 
 def _code(dtype):
@@ -144,7 +162,8 @@ def prefill_workspace(B, T, H, dk, dv, kda, device, stream=None):
     return buf, buf.numel()
 
 
-def _prefill(kda, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream, workspace):
+def _prefill(kda, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream, workspace,
+             prologue=0):
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, d_k]")
     B, T, H, dk = q.shape
@@ -173,34 +192,36 @@ def _prefill(kda, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream
         ws, nws = prefill_workspace(B, T, H, dk, dv, kda, dev, stream)
     else:
         ws, nws = workspace, workspace.numel() * workspace.element_size()
-    fn = lib.kda_prefill if kda else lib.gdn_prefill
+    fn, extra = _pick("kda_prefill" if kda else "gdn_prefill", prologue)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(s0), _ptr(o), _ptr(sf),
               B, T, H, dk, dv, _code(dt), _code(out_dtype), chunk, _ptr(ws), nws,
-              _stream(dev, stream)))
+              _stream(dev, stream), *extra))
     return o, sf
 
 
 def gdn_prefill(q, k, v, alpha, beta, s0=None, *, out_dtype=None, o=None, s_final=None,
-                chunk=CHUNK, stream=None, workspace=None):
+                chunk=CHUNK, stream=None, workspace=None, prologue=0):
     """Gated DeltaNet chunked prefill (scalar gate alpha [B, T, H]).
 
     q, k [B, T, H, d_k] and v [B, T, H, d_v] in float32 or bfloat16; alpha, beta
     float32; s0 [B, H, d_v, d_k] float32 or None.  Returns (o, s_final); pass
     s_final=False to skip writing the final state, or s_final=s0 to carry in place.
+    prologue: PROLOGUE_* flags (raw q, k normalised in the kernel; alpha given as the
+    gate pre-activation x, alpha = exp(-softplus(x))).
     """
     return _prefill(False, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream,
-                    workspace)
+                    workspace, prologue)
 
 
 def kda_prefill(q, k, v, alpha, beta, s0=None, *, out_dtype=None, o=None, s_final=None,
-                chunk=CHUNK, stream=None, workspace=None):
+                chunk=CHUNK, stream=None, workspace=None, prologue=0):
     """Kimi Delta Attention chunked prefill (per-channel gate alpha [B, T, H, d_k]);
     otherwise as ``gdn_prefill``."""
     return _prefill(True, q, k, v, alpha, beta, s0, out_dtype, o, s_final, chunk, stream,
-                    workspace)
+                    workspace, prologue)
 
 
-def _decode(kda, q, k, v, alpha, beta, state, out_dtype, o, stream):
+def _decode(kda, q, k, v, alpha, beta, state, out_dtype, o, stream, prologue=0):
     if q.dim() != 3:
         raise ValueError("q must be [N, H, d_k]")
     N, H, dk = q.shape
@@ -219,25 +240,25 @@ def _decode(kda, q, k, v, alpha, beta, state, out_dtype, o, stream):
     if o is None:
         o = torch.empty((N, H, dv), dtype=out_dtype, device=dev)
     _need(o, "o", (N, H, dv), out_dtype, dev)
-    fn = lib.kda_decode if kda else lib.gdn_decode
+    fn, extra = _pick("kda_decode" if kda else "gdn_decode", prologue)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(o),
-              N, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream)))
+              N, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream), *extra))
     return o
 
 
-def gdn_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
+def gdn_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None, prologue=0):
     """One Gated DeltaNet decode step for N sequences; ``state`` [N, H, d_v, d_k]
     float32 is updated in place.  Returns o [N, H, d_v]."""
-    return _decode(False, q, k, v, alpha, beta, state, out_dtype, o, stream)
+    return _decode(False, q, k, v, alpha, beta, state, out_dtype, o, stream, prologue)
 
 
-def kda_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None):
+def kda_decode(q, k, v, alpha, beta, state, *, out_dtype=None, o=None, stream=None, prologue=0):
     """One Kimi Delta Attention decode step (alpha [N, H, d_k]); as ``gdn_decode``."""
-    return _decode(True, q, k, v, alpha, beta, state, out_dtype, o, stream)
+    return _decode(True, q, k, v, alpha, beta, state, out_dtype, o, stream, prologue)
 
 
 def _prefill_varlen(kda, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
-                    chunk, stream, workspace):
+                    chunk, stream, workspace, prologue=0):
     if q.dim() != 3:
         raise ValueError("q must be [total, H, d_k] (sequences packed along the tokens)")
     total, H, dk = q.shape
@@ -274,34 +295,34 @@ def _prefill_varlen(kda, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dty
         s = stream if stream is not None else torch.cuda.current_stream(dev)
         with torch.cuda.stream(s):
             workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
-    fn = lib.kda_prefill_varlen if kda else lib.gdn_prefill_varlen
+    fn, extra = _pick("kda_prefill_varlen" if kda else "gdn_prefill_varlen", prologue)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens), _ptr(slots),
               _ptr(state), _ptr(o), nseq, total, H, dk, dv, _code(dt), _code(out_dtype), chunk,
-              _ptr(workspace), workspace.numel(), _stream(dev, stream)))
+              _ptr(workspace), workspace.numel(), _stream(dev, stream), *extra))
     return o
 
 
 def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, state, *, slots=None, out_dtype=None,
-                       o=None, chunk=CHUNK, stream=None, workspace=None):
+                       o=None, chunk=CHUNK, stream=None, workspace=None, prologue=0):
     """Gated DeltaNet prefill of nseq sequences packed along the tokens: q, k
     [total, H, d_k], v [total, H, d_v] bf16; alpha, beta [total, H] float32; cu_seqlens
     int32 [nseq + 1] on the device; state a float32 pool [nslots, H, d_v, d_k] read
     from and written back to slot slots[i] (default i) in place.  Returns o."""
     return _prefill_varlen(False, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
-                           chunk, stream, workspace)
+                           chunk, stream, workspace, prologue)
 
 
 def kda_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, state, *, slots=None, out_dtype=None,
-                       o=None, chunk=CHUNK, stream=None, workspace=None):
+                       o=None, chunk=CHUNK, stream=None, workspace=None, prologue=0):
     """Kimi Delta Attention (alpha [total, H, d_k]); as ``gdn_prefill_varlen``."""
     return _prefill_varlen(True, q, k, v, alpha, beta, cu_seqlens, state, slots, out_dtype, o,
-                           chunk, stream, workspace)
+                           chunk, stream, workspace, prologue)
 
 
 VERIFY_MAX_TOKENS = 16
 
 
-def _verify(kda, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream):
+def _verify(kda, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream, prologue=0):
     if q.dim() != 4:
         raise ValueError("q must be [N, K, H, d_k]")
     N, K, H, dk = q.shape
@@ -326,27 +347,30 @@ def _verify(kda, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream):
     if o is None:
         o = torch.empty((N, K, H, dv), dtype=out_dtype, device=dev)
     _need(o, "o", (N, K, H, dv), out_dtype, dev)
-    fn = lib.kda_verify if kda else lib.gdn_verify
+    fn, extra = _pick("kda_verify" if kda else "gdn_verify", prologue)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(snapshots),
-              _ptr(o), N, K, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream)))
+              _ptr(o), N, K, H, dk, dv, _code(dt), _code(out_dtype), _stream(dev, stream),
+              *extra))
     return o, snapshots
 
 
 def gdn_verify(q, k, v, alpha, beta, state, *, snapshots=True, out_dtype=None, o=None,
-               stream=None):
+               stream=None, prologue=0):
     """Gated DeltaNet over K tokens per sequence from a carried state, keeping the
     state after every token.  q, k [N, K, H, d_k]; v [N, K, H, d_v]; alpha, beta
     [N, K, H]; state [N, H, d_v, d_k] float32.  snapshots=True allocates, or pass a
     [K, N, H, d_v, d_k] float32 tensor; snapshots[t] is the state after token t+1 and
     ``state`` is left as it was.  snapshots=False updates ``state`` in place to the
     state after the K tokens instead.  Returns (o [N, K, H, d_v], snapshots or None)."""
-    return _verify(False, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream)
+    return _verify(False, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream,
+                   prologue)
 
 
 def kda_verify(q, k, v, alpha, beta, state, *, snapshots=True, out_dtype=None, o=None,
-               stream=None):
+               stream=None, prologue=0):
     """Kimi Delta Attention (alpha [N, K, H, d_k]); as ``gdn_verify``."""
-    return _verify(True, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream)
+    return _verify(True, q, k, v, alpha, beta, state, snapshots, out_dtype, o, stream,
+                   prologue)
 
 
 def _backward(kda, q, k, v, alpha, beta, s0, do, ds_final, workspace, stream):

@@ -40,6 +40,7 @@ static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Bytes of the status word area at the start of a prefill workspace.
 constexpr size_t kStatusBytes = 256;
+constexpr unsigned kPrologueFlags = GDR_PROLOGUE_L2NORM_QK | GDR_PROLOGUE_GATE_LOGIT;
 
 bool tc_prefill_supported(const PrefillArgs& a);   // prefill_tc.cu
 size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda);
@@ -49,8 +50,9 @@ static gdr_status prefill(bool kda, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, const float* s0, void* o,
                           float* s_final, int B, int T, int H, int dk, int dv, int in_dtype,
                           int out_dtype, int chunk, void* workspace, size_t ws_bytes,
-                          void* stream) {
+                          void* stream, unsigned pro) {
   const char* fn = kda ? "kda_prefill" : "gdn_prefill";
+  if (pro & ~kPrologueFlags) return fail(GDR_ERR_INVALID_ARG, "%s: unknown prologue flags 0x%x", fn, pro);
   if (B < 0 || T < 0 || H < 0)
     return fail(GDR_ERR_INVALID_ARG, "%s: negative size B=%d T=%d H=%d", fn, B, T, H);
   if (!head_ok(dk) || !head_ok(dv))
@@ -89,17 +91,22 @@ static gdr_status prefill(bool kda, const void* q, const void* k, const void* v,
   if ((s0 && !aligned16(s0)) || (s_final && !aligned16(s_final)))
     return fail(GDR_ERR_INVALID_ARG, "%s: s0/s_final not 16-byte aligned", fn);
   PrefillArgs a{q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv,
-                in_dtype, out_dtype, kda, workspace, ws_bytes};
+                in_dtype, out_dtype, kda, workspace, ws_bytes, pro};
   timing_mark(st, -1);
-  cudaError_t e = tc_prefill_supported(a) ? launch_prefill_tc(a, st) : launch_prefill_simt(a, st);
+  // the fused prologue runs in the two-kernel tensor-core prefill or in the CUDA-core
+  // kernel, not in the single-kernel tensor-core fallbacks (used with a small workspace)
+  const bool tc = tc_prefill_supported(a) && (pro == 0 || ws_bytes >= need);
+  cudaError_t e = tc ? launch_prefill_tc(a, st) : launch_prefill_simt(a, st);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return ok();
 }
 
 static gdr_status decode(bool kda, const void* q, const void* k, const void* v,
                          const float* alpha, const float* beta, float* state, void* o, int N,
-                         int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
+                         int H, int dk, int dv, int in_dtype, int out_dtype, void* stream,
+                         unsigned pro) {
   const char* fn = kda ? "kda_decode" : "gdn_decode";
+  if (pro & ~kPrologueFlags) return fail(GDR_ERR_INVALID_ARG, "%s: unknown prologue flags 0x%x", fn, pro);
   if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "%s: negative size N=%d H=%d", fn, N, H);
   if (!head_ok(dk) || !head_ok(dv))
     return fail(GDR_ERR_UNSUPPORTED, "%s: d_k=%d d_v=%d (supported: 32, 64, 128)", fn, dk, dv);
@@ -115,7 +122,7 @@ static gdr_status decode(bool kda, const void* q, const void* k, const void* v,
     if (!aligned16(need_ptrs[i]))
       return fail(GDR_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
   }
-  DecodeArgs a{q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype, kda};
+  DecodeArgs a{q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype, kda, pro};
   cudaError_t e = launch_decode(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return ok();
@@ -124,8 +131,9 @@ static gdr_status decode(bool kda, const void* q, const void* k, const void* v,
 static gdr_status verify(bool kda, const void* q, const void* k, const void* v,
                          const float* alpha, const float* beta, float* state, float* snapshots,
                          void* o, int N, int K, int H, int dk, int dv, int in_dtype,
-                         int out_dtype, void* stream) {
+                         int out_dtype, void* stream, unsigned pro) {
   const char* fn = kda ? "kda_verify" : "gdn_verify";
+  if (pro & ~kPrologueFlags) return fail(GDR_ERR_INVALID_ARG, "%s: unknown prologue flags 0x%x", fn, pro);
   if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "%s: negative size N=%d H=%d", fn, N, H);
   if (K < 1 || K > GDR_VERIFY_MAX_TOKENS)
     return fail(GDR_ERR_UNSUPPORTED, "%s: K=%d tokens (supported: 1 to %d)", fn, K,
@@ -147,7 +155,7 @@ static gdr_status verify(bool kda, const void* q, const void* k, const void* v,
   if (snapshots && !aligned16(snapshots))
     return fail(GDR_ERR_INVALID_ARG, "%s: snapshots is not 16-byte aligned", fn);
   VerifyArgs a{q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv,
-               in_dtype, out_dtype, kda};
+               in_dtype, out_dtype, kda, pro};
   cudaError_t e = launch_verify(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return ok();
@@ -212,7 +220,15 @@ gdr_status gdn_prefill(const void* q, const void* k, const void* v, const float*
                        int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
                        void* workspace, size_t ws_bytes, void* stream) {
   return gdr::prefill(false, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
-                      out_dtype, chunk, workspace, ws_bytes, stream);
+                      out_dtype, chunk, workspace, ws_bytes, stream, 0u);
+}
+
+gdr_status gdn_prefill_ex(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* o, float* s_final, int B,
+                          int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                          void* workspace, size_t ws_bytes, void* stream, unsigned prologue) {
+  return gdr::prefill(false, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
+                      out_dtype, chunk, workspace, ws_bytes, stream, prologue);
 }
 
 gdr_status kda_prefill(const void* q, const void* k, const void* v, const float* alpha,
@@ -220,35 +236,73 @@ gdr_status kda_prefill(const void* q, const void* k, const void* v, const float*
                        int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
                        void* workspace, size_t ws_bytes, void* stream) {
   return gdr::prefill(true, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
-                      out_dtype, chunk, workspace, ws_bytes, stream);
+                      out_dtype, chunk, workspace, ws_bytes, stream, 0u);
+}
+
+gdr_status kda_prefill_ex(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* o, float* s_final, int B,
+                          int T, int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                          void* workspace, size_t ws_bytes, void* stream, unsigned prologue) {
+  return gdr::prefill(true, q, k, v, alpha, beta, s0, o, s_final, B, T, H, dk, dv, in_dtype,
+                      out_dtype, chunk, workspace, ws_bytes, stream, prologue);
 }
 
 gdr_status gdn_decode(const void* q, const void* k, const void* v, const float* alpha,
                       const float* beta, float* state, void* o, int N, int H, int dk, int dv,
                       int in_dtype, int out_dtype, void* stream) {
   return gdr::decode(false, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
-                     stream);
+                     stream, 0u);
+}
+
+gdr_status gdn_decode_ex(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, float* state, void* o, int N, int H, int dk, int dv,
+                         int in_dtype, int out_dtype, void* stream, unsigned prologue) {
+  return gdr::decode(false, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
+                     stream, prologue);
 }
 
 gdr_status kda_decode(const void* q, const void* k, const void* v, const float* alpha,
                       const float* beta, float* state, void* o, int N, int H, int dk, int dv,
                       int in_dtype, int out_dtype, void* stream) {
   return gdr::decode(true, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
-                     stream);
+                     stream, 0u);
+}
+
+gdr_status kda_decode_ex(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, float* state, void* o, int N, int H, int dk, int dv,
+                         int in_dtype, int out_dtype, void* stream, unsigned prologue) {
+  return gdr::decode(true, q, k, v, alpha, beta, state, o, N, H, dk, dv, in_dtype, out_dtype,
+                     stream, prologue);
 }
 
 gdr_status gdn_verify(const void* q, const void* k, const void* v, const float* alpha,
                       const float* beta, float* state, float* snapshots, void* o, int N, int K,
                       int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
   return gdr::verify(false, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
-                     out_dtype, stream);
+                     out_dtype, stream, 0u);
+}
+
+gdr_status gdn_verify_ex(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, float* state, float* snapshots, void* o, int N,
+                         int K, int H, int dk, int dv, int in_dtype, int out_dtype, void* stream,
+                         unsigned prologue) {
+  return gdr::verify(false, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
+                     out_dtype, stream, prologue);
 }
 
 gdr_status kda_verify(const void* q, const void* k, const void* v, const float* alpha,
                       const float* beta, float* state, float* snapshots, void* o, int N, int K,
                       int H, int dk, int dv, int in_dtype, int out_dtype, void* stream) {
   return gdr::verify(true, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
-                     out_dtype, stream);
+                     out_dtype, stream, 0u);
+}
+
+gdr_status kda_verify_ex(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, float* state, float* snapshots, void* o, int N,
+                         int K, int H, int dk, int dv, int in_dtype, int out_dtype, void* stream,
+                         unsigned prologue) {
+  return gdr::verify(true, q, k, v, alpha, beta, state, snapshots, o, N, K, H, dk, dv, in_dtype,
+                     out_dtype, stream, prologue);
 }
 
 size_t gdr_backward_workspace_bytes(int B, int T, int H, int dk, int dv, int kda) {

@@ -49,4 +49,27 @@ __device__ __forceinline__ float log_gate_accurate(float a) {
   return fmaxf(logf(fmaxf(a, 1e-38f)), -GDR_LOG_GATE_FLOOR);
 }
 
+// ---- fused prologue (GDR_PROLOGUE_* flags) --------------------------------------------
+
+// softplus(x) = log(1 + e^x), written so that neither branch overflows
+__device__ __forceinline__ float softplus(float x) {
+  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+// the gate alpha = exp(-softplus(x)) from its pre-activation x
+__device__ __forceinline__ float gate_from_logit(float x) { return expf(-softplus(x)); }
+// log alpha = -softplus(x), floored like log_gate
+__device__ __forceinline__ float log_gate_from_logit(float x) {
+  return fmaxf(-softplus(x), -GDR_LOG_GATE_FLOOR);
+}
+// factor that L2-normalises a vector with this sum of squares
+__device__ __forceinline__ float l2_scale(float sumsq) {
+  return 1.f / sqrtf(sumsq + GDR_L2NORM_EPS);
+}
+// a normalised value as the kernel's input type holds it (bf16 inputs: rounded to bf16)
+template <typename Tin> __device__ __forceinline__ float as_input(float x);
+template <> __device__ __forceinline__ float as_input<float>(float x) { return x; }
+template <> __device__ __forceinline__ float as_input<__nv_bfloat16>(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 }  // namespace gdr

@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
               const Tin* __restrict__ v, const float* __restrict__ alpha,
               const float* __restrict__ beta, float* __restrict__ state,
-              Tout* __restrict__ o, int NH, int dv) {
+              Tout* __restrict__ o, int NH, int dv, unsigned pro) {
   constexpr int LPR = 8;               // lanes per state row
   constexpr int RPW = 32 / LPR;        // rows per warp instruction
   constexpr int F4 = DK / (4 * LPR);   // float4 pieces per lane per row
@@ -52,7 +52,7 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   float kr[F4][4], qr[F4][4], ar[F4][4];
   const Tin* kh = k + head * DK;
   const Tin* qh = q + head * DK;
-  float kq = 0.f;
+  float kq = 0.f, nk = 0.f, nq = 0.f;
 #pragma unroll
   for (int m = 0; m < F4; ++m) {
     const int c = 4 * (j + LPR * m);
@@ -63,14 +63,43 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     if (KDA) {
       float4 aa = *reinterpret_cast<const float4*>(alpha + head * DK + c);
       ar[m][0] = aa.x; ar[m][1] = aa.y; ar[m][2] = aa.z; ar[m][3] = aa.w;
+      if (pro & GDR_PROLOGUE_GATE_LOGIT) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ar[m][e] = gate_from_logit(ar[m][e]);
+      }
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) kq = fmaf(kr[m][e], qr[m][e], kq);
+    for (int e = 0; e < 4; ++e) {
+      nk = fmaf(kr[m][e], kr[m][e], nk);
+      nq = fmaf(qr[m][e], qr[m][e], nq);
+    }
   }
+  if (pro & GDR_PROLOGUE_L2NORM_QK) {
+    // the 8 lanes of a row group hold the whole vectors
+#pragma unroll
+    for (int off = 1; off < LPR; off <<= 1) {
+      nk += __shfl_xor_sync(0xffffffffu, nk, off);
+      nq += __shfl_xor_sync(0xffffffffu, nq, off);
+    }
+    const float sk = l2_scale(nk), sq = l2_scale(nq);
+#pragma unroll
+    for (int m = 0; m < F4; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        kr[m][e] = as_input<Tin>(kr[m][e] * sk);
+        qr[m][e] = as_input<Tin>(qr[m][e] * sq);
+      }
+  }
+#pragma unroll
+  for (int m = 0; m < F4; ++m)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) kq = fmaf(kr[m][e], qr[m][e], kq);
   kq += __shfl_xor_sync(0xffffffffu, kq, 1);
   kq += __shfl_xor_sync(0xffffffffu, kq, 2);
   kq += __shfl_xor_sync(0xffffffffu, kq, 4);
-  const float a_s = KDA ? 1.f : alpha[head];
+  const float a_s = KDA ? 1.f
+                        : ((pro & GDR_PROLOGUE_GATE_LOGIT) ? gate_from_logit(alpha[head])
+                                                           : alpha[head]);
   const float bt = beta[head];
 
   float* Sh = state + head * (long)dv * DK;
@@ -128,11 +157,11 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   if (a.out_dtype == GDR_F32)
     decode_kernel<DK, KDA, Tin, float><<<grid, kDecodeWarps * 32, 0, st>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.beta, a.state,
-        (float*)a.o, NH, a.dv);
+        (float*)a.o, NH, a.dv, a.pro);
   else
     decode_kernel<DK, KDA, Tin, __nv_bfloat16><<<grid, kDecodeWarps * 32, 0, st>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.beta, a.state,
-        (__nv_bfloat16*)a.o, NH, a.dv);
+        (__nv_bfloat16*)a.o, NH, a.dv, a.pro);
   return cudaGetLastError();
 }
 

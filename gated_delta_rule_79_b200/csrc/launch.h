@@ -21,6 +21,7 @@ struct PrefillArgs {
   bool kda;
   void* workspace;
   size_t ws_bytes;
+  unsigned pro;         // GDR_PROLOGUE_* flags (0: q, k normalised and alpha given)
 };
 
 struct DecodeArgs {
@@ -34,6 +35,7 @@ struct DecodeArgs {
   int N, H, dk, dv;
   int in_dtype, out_dtype;
   bool kda;
+  unsigned pro;         // GDR_PROLOGUE_* flags
 };
 
 struct VerifyArgs {
@@ -48,6 +50,7 @@ struct VerifyArgs {
   int N, K, H, dk, dv;
   int in_dtype, out_dtype;
   bool kda;
+  unsigned pro;         // GDR_PROLOGUE_* flags
 };
 
 struct ChunkMap;   // chunkmap.cuh

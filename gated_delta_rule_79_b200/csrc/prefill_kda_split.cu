@@ -80,7 +80,7 @@ constexpr int P_AS = 0, P_XS = 16384, P_ZS = 32768;
 constexpr int P_R = 65536;        // R = K (.) e^{Gm - G}, tf32 [64][128] SW128            32 KB
                                   //   after the Gram: G [64 t][128 c] for wide channels
 constexpr int P_SMALL = P_R + 32768;
-constexpr int P_SMEM = P_SMALL + 3072 + 1024;   // about 100 KB: two CTAs per SM
+constexpr int P_SMEM = P_SMALL + 3584 + 1024;   // about 100 KB: two CTAs per SM
 constexpr uint32_t P_TM_G = 0;    // Gram, M=128 x 64
 constexpr uint32_t P_TM_GS = 64;  // G by channel: lane c, columns t
 constexpr uint32_t P_TM_COLS = 128;
@@ -90,12 +90,14 @@ struct PrepSmall {
   double tot[2][kDK];   // per channel: sum of the log gates of tokens 0-31 and 32-63
   float g0[kDK];        // per channel: G of token 0
   unsigned wmask[4];    // wide channels
+  float rscale[2 * kC]; // fused prologue: the L2 scale of q rows 0-63 and k rows 64-127
   uint32_t tmem;
   unsigned long long mma_bar;
   unsigned long long tma_bar;
 };
-static_assert(sizeof(PrepSmall) <= 3072, "prep small");
+static_assert(sizeof(PrepSmall) <= 3584, "prep small");
 
+template <unsigned PRO>
 __global__ void __launch_bounds__(P_THREADS, 2)
 kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -157,6 +159,41 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (warp == 0) tmem_dealloc(ps.tmem, P_TM_COLS);
       return;
     }
+    if constexpr ((PRO & GDR_PROLOGUE_L2NORM_QK) != 0) {
+      // row tid < 128 of the staged q (0-63) and k (64-127), [t][c] bf16: divided by its
+      // L2 norm in fp32 and rounded back to bf16, in place (threads start at different
+      // 16-byte pieces of their rows, so a warp's reads spread over the banks)
+      if (tid < 2 * kC) {
+        // two passes over the row (sum of squares, then the scaled write-back), so that
+        // no row is held in registers
+        uint4* row = reinterpret_cast<uint4*>(tL + tid * 256);
+        float ss = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const uint4 x = row[(i + tid) & 15];
+          const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hh[e]);
+            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          }
+        }
+        const float sc = l2_scale(ss);
+        ps.rscale[tid] = sc;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          uint4 x = row[(i + tid) & 15];
+          __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hh[e]);
+            hh[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+          }
+          row[(i + tid) & 15] = x;
+        }
+      }
+      __syncthreads();
+    }
     const unsigned short* qs = reinterpret_cast<const unsigned short*>(tL);
     const unsigned short* ks = reinterpret_cast<const unsigned short*>(tL + 16384);
     const float* as = reinterpret_cast<const float*>(tR);
@@ -169,12 +206,18 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
       g[2 * i + 1] = as[(ta + 1) * kDK + cc];
     }
   }
+  constexpr bool kLogit = (PRO & GDR_PROLOGUE_GATE_LOGIT) != 0;
+  if constexpr (kLogit) {
+    // fused prologue: the staged values are the logits x; log alpha = -softplus(x)
+#pragma unroll
+    for (int x = 0; x < 32; ++x) g[x] = log_gate_from_logit(g[x]);
+  }
   // ---- 2. cumulative log gate: fp64 prefix over each half, halves joined by their sums
   {
     double acc = 0.0;
 #pragma unroll
     for (int x = 0; x < 32; ++x) {
-      acc += (32 * hw + x < L) ? (double)log_gate(g[x]) : 0.0;
+      acc += (32 * hw + x < L) ? (double)(kLogit ? g[x] : log_gate(g[x])) : 0.0;
       g[x] = (float)acc;
     }
     ps.tot[hw][cc] = acc;
@@ -294,21 +337,28 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float bt = ps.beta[t];
     tmem_wait_ld();
     if (anywide) {
+      // the exact terms read q, k again from global memory: with the fused prologue they
+      // are normalised here exactly as the staged tile was (same scale, same rounding)
+      constexpr bool nrm = (PRO & GDR_PROLOGUE_L2NORM_QK) != 0;
       const __nv_bfloat16* xs = r < 64 ? q : k;
+      const float xsc = nrm ? ps.rscale[r] : 1.f;
 #pragma unroll 1
       for (int w = 0; w < 4; ++w) {
         unsigned m = ps.wmask[w];
         while (m) {
           const int ch = 32 * w + __ffs(m) - 1;
           m &= m - 1;
-          const float xv = t < L ? __bfloat162float(xs[(row0 + (long)t * H) * kDK + ch]) : 0.f;
+          float xv = t < L ? __bfloat162float(xs[(row0 + (long)t * H) * kDK + ch]) : 0.f;
+          if constexpr (nrm) xv = as_input<__nv_bfloat16>(xv * xsc);
           const float gt = Gw[t * kDK + ch];
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
             const int j = 32 * hw + x;
-            if (j <= t && j < L)
-              d[x] += xv * __bfloat162float(k[(row0 + (long)j * H) * kDK + ch]) *
-                      __expf(gt - Gw[j * kDK + ch]);
+            if (j <= t && j < L) {
+              float kv = __bfloat162float(k[(row0 + (long)j * H) * kDK + ch]);
+              if constexpr (nrm) kv = as_input<__nv_bfloat16>(kv * ps.rscale[kC + j]);
+              d[x] += xv * kv * __expf(gt - Gw[j * kDK + ch]);
+            }
           }
         }
       }
@@ -431,10 +481,11 @@ cudaError_t launch_kda_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStre
       !encode_bthd_f32(&ma, a.alpha, TB, a.T, a.H, kDK, kDK, kC))
     return cudaErrorInvalidValue;
   const uint32_t lim = kda_split_spin_limit();
-  cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  auto prep = a.pro == 3 ? kda_chunk_prep_kernel<3> : a.pro == 2 ? kda_chunk_prep_kernel<2>
+             : a.pro == 1 ? kda_chunk_prep_kernel<1> : kda_chunk_prep_kernel<0>;
+  cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  kda_chunk_prep_kernel<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
+  prep<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
       mq, mk, ma, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.beta,
       (unsigned char*)a.workspace, m, a.H, (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();

@@ -62,7 +62,7 @@ prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                     const Tin* __restrict__ v, const float* __restrict__ alpha,
                     const float* __restrict__ beta, const float* __restrict__ s0,
                     Tout* __restrict__ o, float* __restrict__ s_final,
-                    int T, int H, int dv) {
+                    int T, int H, int dv, unsigned pro) {
   using L = SimtSmem<DK, KDA>;
   extern __shared__ float sm[];
   float* Ks = sm + L::K;    // k, later K (.) e^{G_last - G}
@@ -103,7 +103,10 @@ prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         const long row = ((b * T + t0 + t) * H + h);
         kv = Elem<Tin>::load(k + row * DK + c);
         qv = Elem<Tin>::load(q + row * DK + c);
-        if (KDA) g = log_gate_accurate(alpha[row * DK + c]);
+        if (KDA) {
+          const float a = alpha[row * DK + c];
+          g = (pro & GDR_PROLOGUE_GATE_LOGIT) ? log_gate_from_logit(a) : log_gate_accurate(a);
+        }
       }
       Ks[t * L::LDK + c] = kv;
       Qs[t * L::LDK + c] = qv;
@@ -118,9 +121,37 @@ prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     if (tid < kC) {
       const long row = (b * T + t0 + tid) * H + h;
       Bs[tid] = tid < Lc ? beta[row] : 0.f;
-      if (!KDA) Gs[tid] = tid < Lc ? log_gate_accurate(alpha[row]) : 0.f;
+      if (!KDA) {
+        const float a = tid < Lc ? alpha[row] : 1.f;
+        Gs[tid] = tid >= Lc ? 0.f
+                  : (pro & GDR_PROLOGUE_GATE_LOGIT) ? log_gate_from_logit(a)
+                                                    : log_gate_accurate(a);
+      }
     }
     __syncthreads();
+    if (pro & GDR_PROLOGUE_L2NORM_QK) {
+      // one warp per token row: q and k divided by their L2 norms (fp32), then held as
+      // the input type holds them
+      const int lane = tid & 31;
+      for (int t = tid >> 5; t < Lc; t += kThreads / 32) {
+        float nk = 0.f, nq = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+          nk = fmaf(Ks[t * L::LDK + c], Ks[t * L::LDK + c], nk);
+          nq = fmaf(Qs[t * L::LDK + c], Qs[t * L::LDK + c], nq);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+          nk += __shfl_xor_sync(0xffffffffu, nk, off);
+          nq += __shfl_xor_sync(0xffffffffu, nq, off);
+        }
+        const float sk = l2_scale(nk), sq = l2_scale(nq);
+        for (int c = lane; c < DK; c += 32) {
+          Ks[t * L::LDK + c] = as_input<Tin>(Ks[t * L::LDK + c] * sk);
+          Qs[t * L::LDK + c] = as_input<Tin>(Qs[t * L::LDK + c] * sq);
+        }
+      }
+      __syncthreads();
+    }
     // ---- 2. inclusive cumulative sum of the log gates (fp64, rounded once) --------
     if (KDA) {
       if (tid < DK) {
@@ -264,7 +295,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st) {
   const int grid = a.B * a.H * (a.dv / kDVS);
   kern<<<grid, kThreads, L::BYTES, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                          a.alpha, a.beta, a.s0, (Tout*)a.o, a.s_final,
-                                         a.T, a.H, a.dv);
+                                         a.T, a.H, a.dv, a.pro);
   e = cudaGetLastError();
   if (e == cudaSuccess) timing_mark(st, 0);
   return e;

@@ -97,6 +97,7 @@ struct PrepSmall {
   unsigned long long mma_bar;
 };
 
+template <unsigned PRO>
 __global__ void __launch_bounds__(P_THREADS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ alpha,
@@ -151,7 +152,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
       a = alpha[row];
       bt = beta[row];
     }
-    ps.g[tid] = log_gate_accurate(a);
+    ps.g[tid] = tid >= L ? 0.f
+                : (PRO & GDR_PROLOGUE_GATE_LOGIT) ? log_gate_from_logit(a)
+                                                  : log_gate_accurate(a);
     ps.beta[tid] = bt;
   }
   __syncthreads();
@@ -184,6 +187,38 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) atomicOr(status, 1u);
     if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
     return;
+  }
+  if constexpr ((PRO & GDR_PROLOGUE_L2NORM_QK) != 0) {
+    // row tid of the q/k tile (0-63 q, 64-127 k): divided by its L2 norm in fp32 and
+    // rounded back to bf16, in place, before anything reads it
+    const int r = tid;
+    uint4 x[16];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      x[i] = *reinterpret_cast<const uint4*>(tQK + (i >> 3) * 16384 + r * 128 +
+                                             (((i & 7) ^ (r & 7)) << 4));
+      const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hh[e]);
+        ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+      }
+    }
+    const float sc = l2_scale(ss);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&x[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hh[e]);
+        hh[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+      }
+      *reinterpret_cast<uint4*>(tQK + (i >> 3) * 16384 + r * 128 + (((i & 7) ^ (r & 7)) << 4)) =
+          x[i];
+    }
+    fence_smem_to_async();
+    __syncthreads();
   }
   if (warp == 0) {
     const uint64_t dA = sdesc(aQK, 16, 1024), dB = sdesc(aQK + 8192, 16, 1024);
@@ -400,10 +435,11 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
       !encode_bthd_bf16(&mk, a.k, TB, a.T, a.H, kDK, 64, kC, true))
     return cudaErrorInvalidValue;
   const uint32_t lim = split_spin_limit();
-  cudaError_t e = cudaFuncSetAttribute(gdn_chunk_prep_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  auto prep = a.pro == 3 ? gdn_chunk_prep_kernel<3> : a.pro == 2 ? gdn_chunk_prep_kernel<2>
+             : a.pro == 1 ? gdn_chunk_prep_kernel<1> : gdn_chunk_prep_kernel<0>;
+  cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  gdn_chunk_prep_kernel<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
+  prep<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
       mq, mk, a.alpha, a.beta, (unsigned char*)a.workspace, m, a.H,
       (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();

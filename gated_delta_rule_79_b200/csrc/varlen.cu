@@ -116,8 +116,10 @@ gdr_status prefill_varlen(bool kda, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, const int* cu_seqlens,
                           const int* slots, float* state, void* o, int nseq, int total, int H,
                           int dk, int dv, int in_dtype, int out_dtype, int chunk,
-                          void* workspace, size_t ws_bytes, void* stream) {
+                          void* workspace, size_t ws_bytes, void* stream, unsigned pro) {
   const char* fn = kda ? "kda_prefill_varlen" : "gdn_prefill_varlen";
+  if (pro & ~(GDR_PROLOGUE_L2NORM_QK | GDR_PROLOGUE_GATE_LOGIT))
+    return vfail(GDR_ERR_INVALID_ARG, fn, "unknown prologue flags");
   if (nseq < 0 || total < 0 || H < 0) return vfail(GDR_ERR_INVALID_ARG, fn, "negative size");
   if ((long long)total * H > (1LL << 31) || nseq > (1 << 24))
     return vfail(GDR_ERR_INVALID_ARG, fn, "sizes too large");
@@ -170,7 +172,7 @@ gdr_status prefill_varlen(bool kda, const void* q, const void* k, const void* v,
     m.nck = (int)lay.nck;
     m.img_base = kStatusBytes + lay.idx_bytes;
     PrefillArgs a{q, k, v, alpha, beta, state, o, state, 1, total, H, dk, dv,
-                  in_dtype, out_dtype, kda, workspace, ws_bytes};
+                  in_dtype, out_dtype, kda, workspace, ws_bytes, pro};
     e = kda ? launch_prefill_kda_split(a, m, st) : launch_prefill_split(a, m, st);
   }
   if (e != cudaSuccess) {
@@ -199,7 +201,18 @@ gdr_status gdn_prefill_varlen(const void* q, const void* k, const void* v, const
                               size_t ws_bytes, void* stream) {
   return gdr::prefill_varlen(false, q, k, v, alpha, beta, cu_seqlens, slots, state, o, nseq,
                              total, H, dk, dv, in_dtype, out_dtype, chunk, workspace, ws_bytes,
-                             stream);
+                             stream, 0u);
+}
+
+gdr_status gdn_prefill_varlen_ex(const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, const int* cu_seqlens,
+                                 const int* slots, float* state, void* o, int nseq, int total,
+                                 int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                                 void* workspace, size_t ws_bytes, void* stream,
+                                 unsigned prologue) {
+  return gdr::prefill_varlen(false, q, k, v, alpha, beta, cu_seqlens, slots, state, o, nseq,
+                             total, H, dk, dv, in_dtype, out_dtype, chunk, workspace, ws_bytes,
+                             stream, prologue);
 }
 
 gdr_status kda_prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
@@ -209,7 +222,18 @@ gdr_status kda_prefill_varlen(const void* q, const void* k, const void* v, const
                               size_t ws_bytes, void* stream) {
   return gdr::prefill_varlen(true, q, k, v, alpha, beta, cu_seqlens, slots, state, o, nseq,
                              total, H, dk, dv, in_dtype, out_dtype, chunk, workspace, ws_bytes,
-                             stream);
+                             stream, 0u);
+}
+
+gdr_status kda_prefill_varlen_ex(const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, const int* cu_seqlens,
+                                 const int* slots, float* state, void* o, int nseq, int total,
+                                 int H, int dk, int dv, int in_dtype, int out_dtype, int chunk,
+                                 void* workspace, size_t ws_bytes, void* stream,
+                                 unsigned prologue) {
+  return gdr::prefill_varlen(true, q, k, v, alpha, beta, cu_seqlens, slots, state, o, nseq,
+                             total, H, dk, dv, in_dtype, out_dtype, chunk, workspace, ws_bytes,
+                             stream, prologue);
 }
 
 }  // extern "C"

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
               const float* __restrict__ alpha, const float* __restrict__ beta,
               float* __restrict__ state, float* __restrict__ snaps, Tout* __restrict__ o,
-              int N, int K, int H, int dv) {
+              int N, int K, int H, int dv, unsigned pro) {
   constexpr int LPR = 8;               // lanes per state row
   constexpr int RPW = 32 / LPR;        // rows per warp instruction
   constexpr int F4 = DK / (4 * LPR);   // float4 pieces per lane per row
@@ -53,19 +53,36 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
   for (int t = 0; t < K; ++t) {
     const long row = (n * K + t) * H + h;             // [N, K, H, ...]
     float* tk = ws + t * per_tok;
-    float kq = 0.f;
+    float kq = 0.f, nq = 0.f, nk = 0.f;
     for (int c = lane; c < DK; c += 32) {
       const float qq = Elem<Tin>::load(q + row * DK + c);
       const float kk = Elem<Tin>::load(k + row * DK + c);
       tk[c] = qq;
       tk[DK + c] = kk;
-      if (KDA) tk[2 * DK + c] = alpha[row * DK + c];
-      kq = fmaf(qq, kk, kq);
+      if (KDA) {
+        const float a = alpha[row * DK + c];
+        tk[2 * DK + c] = (pro & GDR_PROLOGUE_GATE_LOGIT) ? gate_from_logit(a) : a;
+      }
+      nq = fmaf(qq, qq, nq);
+      nk = fmaf(kk, kk, nk);
     }
+    if (pro & GDR_PROLOGUE_L2NORM_QK) {
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        nq += __shfl_xor_sync(0xffffffffu, nq, off);
+        nk += __shfl_xor_sync(0xffffffffu, nk, off);
+      }
+      const float sq = l2_scale(nq), sk = l2_scale(nk);
+      for (int c = lane; c < DK; c += 32) {
+        tk[c] = as_input<Tin>(tk[c] * sq);
+        tk[DK + c] = as_input<Tin>(tk[DK + c] * sk);
+      }
+    }
+    for (int c = lane; c < DK; c += 32) kq = fmaf(tk[c], tk[DK + c], kq);
 #pragma unroll
     for (int off = 16; off; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
     if (lane == 0) {
-      if (!KDA) tk[2 * DK] = alpha[row];
+      if (!KDA) tk[2 * DK] = (pro & GDR_PROLOGUE_GATE_LOGIT) ? gate_from_logit(alpha[row]) : alpha[row];
       tk[2 * DK + GA] = beta[row];
       tk[2 * DK + GA + 1] = kq;
     }
@@ -164,14 +181,14 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarps * 32, smem, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                           a.alpha, a.beta, a.state, a.snapshots, (float*)a.o,
-                                          a.N, a.K, a.H, a.dv);
+                                          a.N, a.K, a.H, a.dv, a.pro);
   } else {
     auto kern = verify_kernel<DK, KDA, Tin, __nv_bfloat16>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarps * 32, smem, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                           a.alpha, a.beta, a.state, a.snapshots,
-                                          (__nv_bfloat16*)a.o, a.N, a.K, a.H, a.dv);
+                                          (__nv_bfloat16*)a.o, a.N, a.K, a.H, a.dv, a.pro);
   }
   return cudaGetLastError();
 }

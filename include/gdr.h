@@ -66,6 +66,16 @@ typedef enum gdr_dtype {
 #define GDR_CHUNK 64
 #define GDR_LOG_GATE_FLOOR 30.0f
 
+/* Fused prologue flags of the *_ex entry points (0 = the plain entry points):
+ *   GDR_PROLOGUE_L2NORM_QK  q and k arrive raw; each (token, head) vector is divided
+ *                           by sqrt(sum of its squares + GDR_L2NORM_EPS) in fp32, and
+ *                           with bf16 inputs rounded back to bf16, before use
+ *   GDR_PROLOGUE_GATE_LOGIT the alpha argument holds the gate's pre-activation x, and
+ *                           alpha = exp(-softplus(x)) is formed in the kernel */
+#define GDR_PROLOGUE_L2NORM_QK 1u
+#define GDR_PROLOGUE_GATE_LOGIT 2u
+#define GDR_L2NORM_EPS 1e-6f
+
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 GDR_API int gdr_version(void);
 
@@ -234,6 +244,58 @@ GDR_API gdr_status kda_verify(const void* q, const void* k, const void* v,
                       const float* alpha, const float* beta, float* state, float* snapshots,
                       void* o, int N, int K, int H, int dk, int dv,
                       int in_dtype, int out_dtype, void* stream);
+
+/* Fused prologue.  The configurations draw q and k L2-normalised per (token, head) and
+ * the gates as alpha = exp(-softplus(x)) of a pre-activation x; these variants take the
+ * raw tensors and do that inside the kernels (the pages leave the projections around the
+ * mixer unspecified, so this is the form the configurations imply).  Each has the
+ * arguments of its plain counterpart plus `prologue`, a set of GDR_PROLOGUE_* flags
+ * (0 = the plain call; other bits: GDR_ERR_INVALID_ARG):
+ *   GDR_PROLOGUE_L2NORM_QK   q, k raw (any scale): used as q / sqrt(|q|^2 + 1e-6), the
+ *                            same for k, formed in fp32 and, for bf16 inputs, rounded to
+ *                            bf16 before use
+ *   GDR_PROLOGUE_GATE_LOGIT  alpha holds x (same shape); the gate is exp(-softplus(x))
+ * The bf16 d_k = 128 prefill fuses the prologue into its per-chunk prep kernel when the
+ * workspace has gdr_prefill_workspace_bytes(...) bytes, else runs the CUDA-core kernel
+ * (which fuses it as well); decode and verify fuse it into their kernels. */
+GDR_API gdr_status gdn_prefill_ex(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const float* s0,
+                       void* o, float* s_final, int B, int T, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream, unsigned prologue);
+GDR_API gdr_status kda_prefill_ex(const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const float* s0,
+                       void* o, float* s_final, int B, int T, int H, int dk, int dv,
+                       int in_dtype, int out_dtype, int chunk,
+                       void* workspace, size_t ws_bytes, void* stream, unsigned prologue);
+GDR_API gdr_status gdn_decode_ex(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, void* o,
+                      int N, int H, int dk, int dv, int in_dtype, int out_dtype,
+                      void* stream, unsigned prologue);
+GDR_API gdr_status kda_decode_ex(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state, void* o,
+                      int N, int H, int dk, int dv, int in_dtype, int out_dtype,
+                      void* stream, unsigned prologue);
+GDR_API gdr_status gdn_verify_ex(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state,
+                      float* snapshots, void* o, int N, int K, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream, unsigned prologue);
+GDR_API gdr_status kda_verify_ex(const void* q, const void* k, const void* v,
+                      const float* alpha, const float* beta, float* state,
+                      float* snapshots, void* o, int N, int K, int H, int dk, int dv,
+                      int in_dtype, int out_dtype, void* stream, unsigned prologue);
+GDR_API gdr_status gdn_prefill_varlen_ex(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta,
+                              const int* cu_seqlens, const int* slots, float* state,
+                              void* o, int nseq, int total, int H, int dk, int dv,
+                              int in_dtype, int out_dtype, int chunk, void* workspace,
+                              size_t ws_bytes, void* stream, unsigned prologue);
+GDR_API gdr_status kda_prefill_varlen_ex(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta,
+                              const int* cu_seqlens, const int* slots, float* state,
+                              void* o, int nseq, int total, int H, int dk, int dv,
+                              int in_dtype, int out_dtype, int chunk, void* workspace,
+                              size_t ws_bytes, void* stream, unsigned prologue);
 
 /* Gradients of the mixers.  "Super Apriel: One Checkpoint, Many Speeds", §2B (Training
  * Recipe): the mixers are trained (stochastic distillation, then supervised fine-tuning),

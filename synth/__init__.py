@@ -18,6 +18,8 @@ Workloads (all inputs synthetic; the pages publish no dataset for the mixer):
   kda_varlen    own slot of a state pool ~ 0.02 N(0,1); lengths from varlen_lengths
   gdn_backward  the gradients of the gdn_prefill / kda_prefill shapes; dL/do ~ N(0,1)
   kda_backward  (bf16) and dL/dS_T ~ N(0,1) (fp32), drawn after the inputs
+  *_prologue    gdn_prefill, kda_prefill and decode_gdn with the raw inputs of the fused
+                prologue: q, k not normalised and the gate logits x in place of alpha
 
 Recipe per (batch b, head h) slice, one ``torch.Generator`` (CPU) seeded with
 ``slice_seed(seed, b, h)``, drawing in this fixed order:
@@ -28,6 +30,10 @@ Recipe per (batch b, head h) slice, one ``torch.Generator`` (CPU) seeded with
   beta [T]           = sigmoid(N(0,1))                           (fp32)
   alpha [T] (GDN) or [T, d_k] (KDA) = exp(-softplus(N(0,1) + 2)) (fp32)
   s0 [d_v, d_k]      = 0.02 N(0,1) when the workload has a non-zero state
+
+Prologue workloads draw, in the same order, q and k as N(0,1) times exp(N(0,1)) (one
+scale per vector, drawn after the vector) instead of unit vectors, and the gate logits
+x = N(0,1) + 2 instead of alpha = exp(-softplus(x)).
 
 Stress gate recipes (not part of the workloads; used by tests so that the
 inter-chunk carry matters): "slow" = exp(-softplus(N(0,1) - 5)) (about 0.993),
@@ -59,6 +65,7 @@ class Workload:
     verify: bool = False  # K tokens (the T axis) from a carried state, snapshots kept
     varlen: bool = False  # B sequences of varlen_lengths(w) tokens packed (T: median)
     backward: bool = False  # the gradients of the prefill of these shapes
+    prologue: int = 0       # fused-prologue flags: raw q, k and gate logits are drawn
 
     @property
     def torch_dtype(self):
@@ -85,6 +92,12 @@ WORKLOADS = {
                            varlen=True),
     "gdn_backward": Workload("gdn_backward", "gdn", 1, 32, 4096, 128, 128, "bf16", "zeros",
                              backward=True),
+    "gdn_prefill_prologue": Workload("gdn_prefill_prologue", "gdn", 1, 32, 4096, 128, 128, "bf16",
+                                     "zeros", prologue=3),
+    "kda_prefill_prologue": Workload("kda_prefill_prologue", "kda", 1, 32, 4096, 128, 128, "bf16",
+                                     "zeros", prologue=3),
+    "decode_gdn_prologue": Workload("decode_gdn_prologue", "gdn", 256, 32, 512, 128, 128, "bf16",
+                                    "randn", True, prologue=3),
     "kda_backward": Workload("kda_backward", "kda", 1, 32, 4096, 128, 128, "bf16", "zeros",
                              backward=True),
 }
@@ -128,6 +141,16 @@ def slice_inputs(w: Workload, b: int, h: int, seed: int = 0, gates: str = "workl
     workload dtype; beta [T], alpha [T] or [T, dk] and s0 [dv, dk] (or None) in fp32."""
     g = torch.Generator().manual_seed(slice_seed(seed, b, h))
     T, dk, dv = w.T, w.dk, w.dv
+    if w.prologue:
+        def vec():
+            x = torch.randn((T, dk), generator=g)
+            return (x * torch.exp(torch.randn((T, 1), generator=g))).to(w.torch_dtype)
+        q, k = vec(), vec()
+        v = torch.randn((T, dv), generator=g).to(w.torch_dtype)
+        beta = torch.sigmoid(torch.randn((T,), generator=g))
+        alpha = torch.randn((T, dk) if w.mixer == "kda" else (T,), generator=g) + 2.0
+        s0 = 0.02 * torch.randn((dv, dk), generator=g) if w.state == "randn" else None
+        return dict(q=q, k=k, v=v, beta=beta, alpha=alpha, s0=s0)
     q = _unit_rows(torch.randn((T, dk), generator=g)).to(w.torch_dtype)
     k = _unit_rows(torch.randn((T, dk), generator=g)).to(w.torch_dtype)
     v = torch.randn((T, dv), generator=g).to(w.torch_dtype)
@@ -177,6 +200,9 @@ def device_inputs(w: Workload, device, seed: int = 0, dtype_override=None):
 
     def unit(shape):
         x = torch.randn(shape, generator=g, device=device)
+        if w.prologue:
+            scale = torch.exp(torch.randn(shape[:-1] + (1,), generator=g, device=device))
+            return (x * scale).to(dt)
         return (x / x.norm(dim=-1, keepdim=True)).to(dt)
 
     q = unit(lead + (dk,))
@@ -184,7 +210,8 @@ def device_inputs(w: Workload, device, seed: int = 0, dtype_override=None):
     v = torch.randn(lead + (dv,), generator=g, device=device).to(dt)
     beta = torch.sigmoid(torch.randn(lead, generator=g, device=device))
     ashape = lead + (dk,) if w.mixer == "kda" else lead
-    alpha = torch.exp(-F.softplus(torch.randn(ashape, generator=g, device=device) + 2.0))
+    logit = torch.randn(ashape, generator=g, device=device) + 2.0
+    alpha = logit if w.prologue else torch.exp(-F.softplus(logit))
     s0 = None
     if w.state == "randn":
         s0 = 0.02 * torch.randn((B, H, dv, dk), generator=g, device=device)
