@@ -15,20 +15,21 @@
 //   dalpha_t[c] = sum_r S_{t-1}[r, c] dS~[r, c];  dS <- dS~ Diag(alpha_t)
 //
 // Every row r of S (a value channel) evolves on its own, forward and in reverse; only
-// dq, dk, dalpha and dbeta sum over rows.  So one warp owns one value row (each lane
-// d_k / 32 key channels), a CTA owns 16 rows, and the d_v / 16 CTAs of one (sequence,
-// head) form a thread-block cluster that sums the per-row terms through distributed
-// shared memory.
+// dq, dk, dalpha and dbeta sum over rows.  So a warp owns two value rows (each lane
+// d_k / 32 key channels of both), a CTA of 16 warps owns 32 rows, and the d_v / 32
+// CTAs of one (sequence, head) form a thread-block cluster that sums the per-row terms
+// through distributed shared memory.
 //
 // Pass 1 runs the recurrence forward and leaves, in the workspace, the state entering
-// every chunk of 64 tokens and u_t, r_t of every token.  Pass 2 walks the chunks in
-// reverse: from the chunk's entering state it rebuilds the states (no reductions: u_t is
-// known) at every eighth token, then in blocks of eight tokens (their states in
-// registers) runs the reverse steps.  The per-row terms of a token are summed over the
-// CTA's warps in shared memory, and those of each block of eight tokens over the
-// cluster's CTAs, which write the results.  Everything is fp32; there is no wait on
-// another CTA other than the cluster barrier, which every CTA of a cluster reaches the
-// same number of times.
+// every segment of 32 tokens and u_t, r_t of every token.  Pass 2 walks the segments in
+// reverse: from the segment's entering state it rebuilds the state at every eighth token
+// (no reductions: u_t is known; four states kept), then in blocks of four tokens (their
+// states in registers, rebuilt from the nearest of those) runs the reverse steps.  Each
+// warp leaves its rows' terms of the block's four tokens in shared memory; one barrier
+// later the CTA sums them over its warps, and one cluster barrier later the cluster's
+// CTAs sum those and write the results.  Everything is fp32; there is no wait on another
+// CTA other than the cluster barrier, which every CTA of a cluster reaches the same
+// number of times.
 
 #include <stdio.h>
 #include <stdint.h>
@@ -40,38 +41,43 @@
 namespace gdr {
 namespace {
 
-constexpr int kC = GDR_CHUNK;
-constexpr int BW_ROWS = 16;            // value rows per CTA, one per warp
-constexpr int BW_THREADS = 32 * BW_ROWS;
-constexpr int BW_BLOCK = 8;            // tokens per reverse block (states in registers)
+constexpr int BW_WARPS = 16;
+constexpr int BW_RPW = 2;                       // value rows per warp
+constexpr int BW_ROWS = BW_WARPS * BW_RPW;      // value rows per CTA
+constexpr int BW_THREADS = 32 * BW_WARPS;
+constexpr int BW_SEG = 32;                      // tokens per staged segment (checkpointed)
+constexpr int BW_SUB = 8;                       // tokens between rebuilt states
+constexpr int BW_BLOCK = 4;                     // tokens per reverse block
+constexpr int BW_NSUB = BW_SEG / BW_SUB;
 
 template <int DK, bool KDA>
 struct BwCfg {
-  static constexpr int NC = DK / 32;                    // key channels per lane
-  static constexpr int NQ = KDA ? 3 * DK + 1 : 2 * DK + 2;   // per-token sums
-  // dq at [0, DK), dk at [DK, 2 DK), dalpha at [2 DK, 2 DK + (KDA ? DK : 1)), dbeta last
-  static constexpr int NA = KDA ? DK : 1;
+  static constexpr int NC = DK / 32;                         // key channels per lane
+  static constexpr int NA = KDA ? DK : 1;                    // gate floats per token
+  // per-token sums: dq at [0, DK), dk at [DK, 2 DK), dalpha at [2 DK, 2 DK + NA), dbeta
+  static constexpr int NQ = 2 * DK + NA + 1;
 };
 
 template <int DK, bool KDA, typename Tin>
 struct BwSmem {
   static constexpr int NQ = BwCfg<DK, KDA>::NQ;
-  Tin k[kC][DK];
-  Tin q[kC][DK];
-  float alpha[kC][BwCfg<DK, KDA>::NA];
-  float beta[kC];
-  float v[kC][BW_ROWS];
-  float dO[kC][BW_ROWS];
-  float u[kC][BW_ROWS];
-  float res[kC][BW_ROWS];
-  float scratch[2][BW_ROWS][NQ];                // per-warp terms, by token parity
-  float part[2][BW_BLOCK][NQ];                  // the CTA's terms, by block parity
+  Tin k[BW_SEG][DK];
+  Tin q[BW_SEG][DK];
+  float alpha[BW_SEG][BwCfg<DK, KDA>::NA];
+  float beta[BW_SEG];
+  float vd[BW_SEG][BW_ROWS];                    // v (pass 1), dL/do (pass 2)
+  float u[BW_SEG][BW_ROWS];
+  float res[BW_SEG][BW_ROWS];
+  float scratch[BW_BLOCK][BW_WARPS][NQ];        // each warp's terms of the block's tokens
+  float part[2][BW_BLOCK][NQ];                  // the CTA's sums, by block parity
 };
 
-__device__ __forceinline__ float warp_sum(float x) {
+__device__ __forceinline__ void warp_sum2(float& a, float& b) {
 #pragma unroll
-  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+  for (int o = 16; o; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
 }
 
 __device__ __forceinline__ void cluster_sync() {
@@ -85,12 +91,15 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-// fp32 at the same shared-memory offset in CTA `rank` of the cluster
-__device__ __forceinline__ float ld_cluster(const float* local, uint32_t rank) {
+// shared-memory address of the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const float* local, uint32_t rank) {
   uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local)), ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  return ra;
+}
+__device__ __forceinline__ float ld_cluster(uint32_t addr) {
   float x;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(ra) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(addr));
   return x;
 }
 
@@ -115,52 +124,49 @@ gdr_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   const int bh = blockIdx.x / ncl;
   const int h = bh % H, b = bh / H;
   const uint32_t crank = cluster_rank();          // == rb: clusters are ncl consecutive CTAs
-  const int r = rb * BW_ROWS + warp;              // this warp's value row
-  const int nchunks = (T + kC - 1) / kC;
-  // workspace of this CTA: entering states [nchunks][16][DK], then u, r [nchunks][2][64][16]
-  float* ckpt = ws + (size_t)blockIdx.x * ((size_t)nchunks * BW_ROWS * (DK + 2 * kC));
-  float* ures = ckpt + (size_t)nchunks * BW_ROWS * DK;
-  const long row_stride = (long)H;                // tokens: ((b T + t) H + h) * width
+  const int r0 = rb * BW_ROWS + BW_RPW * warp;    // this warp's first value row
+  const int rl = BW_RPW * warp;                   // ... within the CTA
+  const int nseg = (T + BW_SEG - 1) / BW_SEG;
+  // workspace of this CTA: entering states [nseg][32 rows][DK], then u, r [nseg][2][32][32]
+  float* ckpt = ws + (size_t)blockIdx.x * ((size_t)nseg * BW_ROWS * (DK + 2 * BW_SEG));
+  float* ures = ckpt + (size_t)nseg * BW_ROWS * DK;
+  auto tok = [&](int t) -> long { return ((long)b * T + t) * H + h; };   // token row index
 
-  // ---- chunk inputs into shared memory (tokens past T: k = q = 0, alpha = 1, beta = 0) ---
-  auto load_chunk = [&](int c, bool reverse_pass) {
-    const int t0 = c * kC;
-    const int L = min(kC, T - t0);
-    constexpr int VEC = 16 / sizeof(Tin);         // elements per 16-byte piece
-    constexpr int PR = DK / VEC;                  // pieces per token row
-    for (int i = tid; i < kC * PR; i += BW_THREADS) {
+  // ---- one segment's inputs into shared memory (tokens past T: zeros, alpha 1, beta 0) ---
+  auto load_seg = [&](int sg, bool reverse_pass) {
+    const int t0 = sg * BW_SEG;
+    const int L = min(BW_SEG, T - t0);
+    constexpr int VEC = 16 / sizeof(Tin);
+    constexpr int PR = DK / VEC;
+    for (int i = tid; i < BW_SEG * PR; i += BW_THREADS) {
       const int t = i / PR, p = i - t * PR;
       uint4 x = make_uint4(0, 0, 0, 0), y = make_uint4(0, 0, 0, 0);
       if (t < L) {
-        const long off = (((long)b * T + t0 + t) * row_stride + h) * DK + p * VEC;
+        const long off = tok(t0 + t) * DK + p * VEC;
         x = *reinterpret_cast<const uint4*>(k + off);
         if (reverse_pass) y = *reinterpret_cast<const uint4*>(q + off);
       }
       *reinterpret_cast<uint4*>(&sm.k[t][p * VEC]) = x;
       if (reverse_pass) *reinterpret_cast<uint4*>(&sm.q[t][p * VEC]) = y;
     }
-    for (int i = tid; i < kC * NA; i += BW_THREADS) {
-      const int t = i / NA, cc = i - t * NA;
-      float a = 1.f;
-      if (t < L) a = alpha[(((long)b * T + t0 + t) * row_stride + h) * NA + cc];
-      sm.alpha[t][cc] = a;
+    for (int i = tid; i < BW_SEG * NA; i += BW_THREADS) {
+      const int t = i / NA, c = i - t * NA;
+      sm.alpha[t][c] = t < L ? alpha[tok(t0 + t) * NA + c] : 1.f;
     }
-    for (int i = tid; i < kC * BW_ROWS; i += BW_THREADS) {
+    for (int i = tid; i < BW_SEG * BW_ROWS; i += BW_THREADS) {
       const int t = i / BW_ROWS, rr = i - t * BW_ROWS;
-      float x = 0.f, y = 0.f;
+      float x = 0.f;
       if (t < L) {
-        const long off = (((long)b * T + t0 + t) * row_stride + h) * DV + rb * BW_ROWS + rr;
-        x = Elem<Tin>::load(v + off);
-        if (reverse_pass) y = Elem<Tdo>::load(dO + off);
+        const long off = tok(t0 + t) * DV + rb * BW_ROWS + rr;
+        x = reverse_pass ? Elem<Tdo>::load(dO + off) : Elem<Tin>::load(v + off);
       }
-      sm.v[t][rr] = x;
+      sm.vd[t][rr] = x;
       if (reverse_pass) {
-        sm.dO[t][rr] = y;
-        sm.u[t][rr] = t < L ? ures[((size_t)c * 2 + 0) * kC * BW_ROWS + i] : 0.f;
-        sm.res[t][rr] = t < L ? ures[((size_t)c * 2 + 1) * kC * BW_ROWS + i] : 0.f;
+        sm.u[t][rr] = t < L ? ures[((size_t)sg * 2 + 0) * BW_SEG * BW_ROWS + i] : 0.f;
+        sm.res[t][rr] = t < L ? ures[((size_t)sg * 2 + 1) * BW_SEG * BW_ROWS + i] : 0.f;
       }
     }
-    if (tid < kC) sm.beta[tid] = tid < L ? beta[((long)b * T + t0 + tid) * row_stride + h] : 0.f;
+    if (tid < BW_SEG) sm.beta[tid] = tid < L ? beta[tok(t0 + tid)] : 0.f;
   };
   auto ld_k = [&](int t, float (&x)[NC]) {
 #pragma unroll
@@ -174,162 +180,226 @@ gdr_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 #pragma unroll
     for (int j = 0; j < NC; ++j) x[j] = KDA ? sm.alpha[t][(lane + 32 * j) % NA] : sm.alpha[t][0];
   };
+  // S <- S Diag(alpha_t) + u_t k_t^T for this warp's two rows (u_t known)
+  auto step_known = [&](int t, float (&S)[BW_RPW][NC]) {
+    float kk[NC], aa[NC];
+    ld_k(t, kk);
+    ld_a(t, aa);
+#pragma unroll
+    for (int p = 0; p < BW_RPW; ++p) {
+      const float uu = sm.u[t][rl + p];
+#pragma unroll
+      for (int j = 0; j < NC; ++j) S[p][j] = fmaf(uu, kk[j], S[p][j] * aa[j]);
+    }
+  };
 
   // =============================== pass 1: forward ======================================
-  float S[NC];
-  {
-    const long srow = (((long)b * H + h) * DV + r) * DK;
+  float S[BW_RPW][NC];
 #pragma unroll
-    for (int j = 0; j < NC; ++j) S[j] = s0 ? s0[srow + lane + 32 * j] : 0.f;
+  for (int p = 0; p < BW_RPW; ++p) {
+    const long srow = (((long)b * H + h) * DV + r0 + p) * DK;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) S[p][j] = s0 ? s0[srow + lane + 32 * j] : 0.f;
   }
-  for (int c = 0; c < nchunks; ++c) {
-    const int L = min(kC, T - c * kC);
+  for (int sg = 0; sg < nseg; ++sg) {
+    const int L = min(BW_SEG, T - sg * BW_SEG);
 #pragma unroll
-    for (int j = 0; j < NC; ++j) ckpt[((size_t)c * BW_ROWS + warp) * DK + lane + 32 * j] = S[j];
-    __syncthreads();                              // the previous chunk's inputs are read
-    load_chunk(c, false);
+    for (int p = 0; p < BW_RPW; ++p)
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        ckpt[((size_t)sg * BW_ROWS + rl + p) * DK + lane + 32 * j] = S[p][j];
+    __syncthreads();                              // the previous segment's inputs are read
+    load_seg(sg, false);
     __syncthreads();
     for (int t = 0; t < L; ++t) {
-      float kk[NC], aa[NC], a = 0.f;
+      float kk[NC], aa[NC], a0 = 0.f, a1 = 0.f;
       ld_k(t, kk);
       ld_a(t, aa);
 #pragma unroll
       for (int j = 0; j < NC; ++j) {
-        S[j] *= aa[j];
-        a = fmaf(S[j], kk[j], a);
+        S[0][j] *= aa[j];
+        S[1][j] *= aa[j];
+        a0 = fmaf(S[0][j], kk[j], a0);
+        a1 = fmaf(S[1][j], kk[j], a1);
       }
-      a = warp_sum(a);
-      const float rr = sm.v[t][warp] - a, uu = sm.beta[t] * rr;
+      warp_sum2(a0, a1);
+      const float bt = sm.beta[t];
+      const float q0 = sm.vd[t][rl] - a0, q1 = sm.vd[t][rl + 1] - a1;
+      const float u0 = bt * q0, u1 = bt * q1;
 #pragma unroll
-      for (int j = 0; j < NC; ++j) S[j] = fmaf(uu, kk[j], S[j]);
-      if (lane == 0) {
-        ures[((size_t)c * 2 + 0) * kC * BW_ROWS + t * BW_ROWS + warp] = uu;
-        ures[((size_t)c * 2 + 1) * kC * BW_ROWS + t * BW_ROWS + warp] = rr;
+      for (int j = 0; j < NC; ++j) {
+        S[0][j] = fmaf(u0, kk[j], S[0][j]);
+        S[1][j] = fmaf(u1, kk[j], S[1][j]);
       }
+      if (lane < 2) {
+        sm.u[t][rl + lane] = lane ? u1 : u0;
+        sm.res[t][rl + lane] = lane ? q1 : q0;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < L * BW_ROWS; i += BW_THREADS) {
+      const int t = i / BW_ROWS, rr = i - t * BW_ROWS;
+      ures[((size_t)sg * 2 + 0) * BW_SEG * BW_ROWS + i] = sm.u[t][rr];
+      ures[((size_t)sg * 2 + 1) * BW_SEG * BW_ROWS + i] = sm.res[t][rr];
     }
   }
   __syncthreads();
-  __threadfence_block();
 
   // =============================== pass 2: reverse ======================================
-  float dS[NC];
-  {
-    const long srow = (((long)b * H + h) * DV + r) * DK;
+  float dS[BW_RPW][NC];
 #pragma unroll
-    for (int j = 0; j < NC; ++j) dS[j] = ds_final ? ds_final[srow + lane + 32 * j] : 0.f;
+  for (int p = 0; p < BW_RPW; ++p) {
+    const long srow = (((long)b * H + h) * DV + r0 + p) * DK;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) dS[p][j] = ds_final ? ds_final[srow + lane + 32 * j] : 0.f;
   }
-  int sp = 0, pb = 0;                             // token parity (scratch), block parity (part)
-  float sub[kC / BW_BLOCK][NC];                   // the state before every eighth token
-  for (int c = nchunks - 1; c >= 0; --c) {
-    const int t0 = c * kC;
-    const int L = min(kC, T - t0);
+  int pb = 0;                                     // block parity (part)
+  for (int sg = nseg - 1; sg >= 0; --sg) {
+    const int t0 = sg * BW_SEG;
+    const int L = min(BW_SEG, T - t0);
     __syncthreads();
-    load_chunk(c, true);
+    load_seg(sg, true);
     __syncthreads();
+    // the state before tokens 0, 8, 16, 24 of the segment
+    float sub[BW_NSUB][BW_RPW][NC];
     {
-      float Sx[NC];
+      float Sx[BW_RPW][NC];
 #pragma unroll
-      for (int j = 0; j < NC; ++j) Sx[j] = ckpt[((size_t)c * BW_ROWS + warp) * DK + lane + 32 * j];
-      for (int s = 0; s < kC / BW_BLOCK; ++s) {
+      for (int p = 0; p < BW_RPW; ++p)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) sub[s][j] = Sx[j];
-        for (int t = s * BW_BLOCK; t < min(L, (s + 1) * BW_BLOCK); ++t) {
-          float kk[NC], aa[NC];
-          ld_k(t, kk);
-          ld_a(t, aa);
-          const float uu = sm.u[t][warp];
+        for (int j = 0; j < NC; ++j)
+          Sx[p][j] = ckpt[((size_t)sg * BW_ROWS + rl + p) * DK + lane + 32 * j];
 #pragma unroll
-          for (int j = 0; j < NC; ++j) Sx[j] = fmaf(uu, kk[j], Sx[j] * aa[j]);
-        }
+      for (int s = 0; s < BW_NSUB; ++s) {
+#pragma unroll
+        for (int p = 0; p < BW_RPW; ++p)
+#pragma unroll
+          for (int j = 0; j < NC; ++j) sub[s][p][j] = Sx[p][j];
+        if (s + 1 < BW_NSUB)
+          for (int t = s * BW_SUB; t < (s + 1) * BW_SUB; ++t) step_known(t, Sx);
       }
     }
-    const int nblk = (L + BW_BLOCK - 1) / BW_BLOCK;
-    for (int s = nblk - 1; s >= 0; --s) {
-      const int tb = s * BW_BLOCK;
-      // states before tokens tb .. tb + 7
-      float blk[BW_BLOCK][NC];
+    // blocks of four tokens, last first; block n covers tokens 4n .. 4n + 3
 #pragma unroll
-      for (int j = 0; j < NC; ++j) blk[0][j] = sub[s][j];
+    for (int nn = 0; nn < BW_SEG / BW_BLOCK; ++nn) {
+      const int n = BW_SEG / BW_BLOCK - 1 - nn;
+      const int tb = n * BW_BLOCK;
+      if (tb >= L) continue;                      // uniform over the cluster
+      // states before tokens tb .. tb + 3, rebuilt from the state before token 8 (n / 2)
+      float blk[BW_BLOCK][BW_RPW][NC];
+      {
+        float Sx[BW_RPW][NC];
 #pragma unroll
-      for (int i = 1; i < BW_BLOCK; ++i) {
-        const int t = tb + i - 1;
-        float kk[NC], aa[NC];
-        ld_k(t, kk);
-        ld_a(t, aa);
-        const float uu = sm.u[t][warp];
+        for (int p = 0; p < BW_RPW; ++p)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) blk[i][j] = fmaf(uu, kk[j], blk[i - 1][j] * aa[j]);
+          for (int j = 0; j < NC; ++j) Sx[p][j] = sub[n / 2][p][j];
+        if (n & 1)
+#pragma unroll
+          for (int t = tb - BW_BLOCK; t < tb; ++t) step_known(t, Sx);
+#pragma unroll
+        for (int i = 0; i < BW_BLOCK; ++i) {
+#pragma unroll
+          for (int p = 0; p < BW_RPW; ++p)
+#pragma unroll
+            for (int j = 0; j < NC; ++j) blk[i][p][j] = Sx[p][j];
+          if (i + 1 < BW_BLOCK) step_known(tb + i, Sx);
+        }
       }
 #pragma unroll
       for (int ii = 0; ii < BW_BLOCK; ++ii) {
         const int i = BW_BLOCK - 1 - ii;
         const int t = tb + i;
-        if (t >= L) continue;                     // uniform over the CTA
+        float* sc = sm.scratch[i][warp];
+        if (t >= L) {                             // past the end: no terms
+          for (int x = lane; x < NQ; x += 32) sc[x] = 0.f;
+          continue;
+        }
         float kk[NC], qq[NC], aa[NC];
         ld_k(t, kk);
         ld_q(t, qq);
         ld_a(t, aa);
-        const float uu = sm.u[t][warp], rr = sm.res[t][warp], bt = sm.beta[t];
-        const float od = sm.dO[t][warp];
-        float Sd[NC], du = 0.f;
+        const float bt = sm.beta[t];
+        float uu[BW_RPW], od[BW_RPW], rr[BW_RPW], du[BW_RPW];
 #pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          Sd[j] = blk[i][j] * aa[j];                   // S~
-          dS[j] = fmaf(od, qq[j], dS[j]);              // + do q^T
-          du = fmaf(dS[j], kk[j], du);
+        for (int p = 0; p < BW_RPW; ++p) {
+          uu[p] = sm.u[t][rl + p];
+          od[p] = sm.vd[t][rl + p];
+          rr[p] = sm.res[t][rl + p];
+          du[p] = 0.f;
         }
-        du = warp_sum(du);
-        float* sc = sm.scratch[sp][warp];
+#pragma unroll
+        for (int p = 0; p < BW_RPW; ++p)
+#pragma unroll
+          for (int j = 0; j < NC; ++j) {
+            dS[p][j] = fmaf(od[p], qq[j], dS[p][j]);           // + do q^T
+            du[p] = fmaf(dS[p][j], kk[j], du[p]);
+          }
+        warp_sum2(du[0], du[1]);
         float ga = 0.f;
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
           const int cc = lane + 32 * j;
-          const float St = fmaf(uu, kk[j], Sd[j]);     // S_t
-          const float dSd = fmaf(-bt * du, kk[j], dS[j]);
-          sc[cc] = St * od;                                        // dq
-          sc[DK + cc] = fmaf(dS[j], uu, -bt * Sd[j] * du);         // dk
-          const float g = blk[i][j] * dSd;                         // dalpha
-          if constexpr (KDA) sc[2 * DK + cc] = g;
-          else ga += g;
-          dS[j] = dSd * aa[j];
+          float pq = 0.f, pk = 0.f, pa = 0.f;
+#pragma unroll
+          for (int p = 0; p < BW_RPW; ++p) {
+            const float Sd = blk[i][p][j] * aa[j];             // S~
+            const float St = fmaf(uu[p], kk[j], Sd);           // S_t
+            const float dSd = fmaf(-bt * du[p], kk[j], dS[p][j]);
+            pq = fmaf(St, od[p], pq);                          // dq
+            pk = fmaf(dS[p][j], uu[p], fmaf(-bt * du[p], Sd, pk));   // dk
+            pa = fmaf(blk[i][p][j], dSd, pa);                  // dalpha
+            dS[p][j] = dSd * aa[j];
+          }
+          sc[cc] = pq;
+          sc[DK + cc] = pk;
+          if constexpr (KDA) sc[2 * DK + cc] = pa;
+          else ga += pa;
         }
-        if constexpr (!KDA) ga = warp_sum(ga);
+        if constexpr (!KDA) {
+#pragma unroll
+          for (int o = 16; o; o >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, o);
+        }
         if (lane == 0) {
           if constexpr (!KDA) sc[2 * DK] = ga;
-          sc[NQ - 1] = du * rr;                                    // dbeta
-          dv[(((long)b * T + t0 + t) * row_stride + h) * DV + r] = bt * du;
+          sc[NQ - 1] = du[0] * rr[0] + du[1] * rr[1];          // dbeta
         }
-        __syncthreads();
-        for (int x = tid; x < NQ; x += BW_THREADS) {
-          float acc = 0.f;
-#pragma unroll
-          for (int w = 0; w < BW_ROWS; ++w) acc += sm.scratch[sp][w][x];
-          sm.part[pb][i][x] = acc;
-        }
-        sp ^= 1;
+        if (lane < BW_RPW)
+          dv[tok(t0 + t) * DV + r0 + lane] = bt * (lane ? du[1] : du[0]);
       }
-      // ---- the block's sums over the cluster's CTAs, written out -------------------------
+      // ---- the block's sums: over the CTA's warps, then over the cluster's CTAs ---------
+      __syncthreads();
+      for (int x = tid; x < BW_BLOCK * NQ; x += BW_THREADS) {
+        const int i = x / NQ, y = x - i * NQ;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < BW_WARPS; ++w) acc += sm.scratch[i][w][y];
+        sm.part[pb][i][y] = acc;
+      }
       cluster_sync();
       for (int i = crank; i < BW_BLOCK; i += ncl) {
         const int t = tb + i;
         if (t >= L) continue;
-        const long tok = ((long)b * T + t0 + t) * row_stride + h;
+        const long tr = tok(t0 + t);
         for (int x = tid; x < NQ; x += BW_THREADS) {
-          float acc = 0.f;
-          for (int rk = 0; rk < ncl; ++rk) acc += ld_cluster(&sm.part[pb][i][x], (uint32_t)rk);
-          if (x < DK) dq[tok * DK + x] = acc;
-          else if (x < 2 * DK) dk[tok * DK + x - DK] = acc;
-          else if (x < 2 * DK + NA) dalpha[tok * NA + x - 2 * DK] = acc;
-          else if (x == NQ - 1) dbeta[tok] = acc;
+          float got[4];
+#pragma unroll
+          for (int rk = 0; rk < 4; ++rk)
+            got[rk] = rk < ncl ? ld_cluster(cluster_addr(&sm.part[pb][i][x], (uint32_t)rk)) : 0.f;
+          const float acc = (got[0] + got[1]) + (got[2] + got[3]);
+          if (x < DK) dq[tr * DK + x] = acc;
+          else if (x < 2 * DK) dk[tr * DK + x - DK] = acc;
+          else if (x < 2 * DK + NA) dalpha[tr * NA + x - 2 * DK] = acc;
+          else dbeta[tr] = acc;
         }
       }
       pb ^= 1;
     }
   }
-  {
-    const long srow = (((long)b * H + h) * DV + r) * DK;
 #pragma unroll
-    for (int j = 0; j < NC; ++j) ds0[srow + lane + 32 * j] = dS[j];
+  for (int p = 0; p < BW_RPW; ++p) {
+    const long srow = (((long)b * H + h) * DV + r0 + p) * DK;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) ds0[srow + lane + 32 * j] = dS[p][j];
   }
   cluster_sync();                                 // no CTA leaves while others read its sums
 }
@@ -339,8 +409,6 @@ cudaError_t launch_bw(const BackwardArgs& a, cudaStream_t st) {
   auto kern = gdr_backward_kernel<DK, KDA, Tin, Tdo>;
   const int smem = (int)sizeof(BwSmem<DK, KDA, Tin>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   if (e != cudaSuccess) return e;
   const int ncl = a.dv / BW_ROWS;
   cudaLaunchConfig_t cfg = {};
@@ -381,8 +449,8 @@ cudaError_t launch_bw_types(const BackwardArgs& a, cudaStream_t st) {
 }  // namespace
 
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
-  const size_t nchunks = ((size_t)T + kC - 1) / kC;
-  return (size_t)B * H * nchunks * dv * (dk + 2 * kC) * sizeof(float);
+  const size_t nseg = ((size_t)T + BW_SEG - 1) / BW_SEG;
+  return (size_t)B * H * nseg * dv * (dk + 2 * BW_SEG) * sizeof(float);
 }
 
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
