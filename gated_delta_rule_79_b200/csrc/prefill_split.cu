@@ -11,13 +11,10 @@
 //   S^T <- e^{G_last} S0^T + K^T Diag(e^{G_last-G}) U
 //
 // Everything but the state-dependent products is computed by gdn_chunk_prep_kernel
-// for every chunk of every head at once (the whole GPU works on them in parallel):
-// the Gram [Q; K] K^T runs as one exact kind::f16 product on the bf16 q, k tiles (the
-// scalar decays e^{G_t - G_j} are applied on read-back), then the triangular solve
-// gives T.  It leaves the chunk's operand images for the carry in the workspace
-// (chunk_image.cuh): [Q (.) e^G; K (.) e^G], e^{G_last}, T, (K (.) e^{G_last - G})^T and
-// P as tf32 tiles.  The state carry that walks the chunks in order is shared with KDA
-// (carry_rows.cu, carry_sliced.cu).
+// for every chunk of every head at once (the whole GPU works on them in parallel; the
+// per-chunk work is gdn_prep.cuh).  It leaves the chunk's operand images for the carry
+// in the workspace (chunk_image.cuh).  The state carry that walks the chunks in order is
+// shared with KDA (carry_rows.cu, carry_sliced.cu).
 //
 // Precision: the Gram is exact (bf16 inputs, fp32 accumulation); the carry's products
 // run as kind::tf32 with operands rounded to nearest.  Waits are bounded; a give-up
@@ -26,79 +23,18 @@
 #include <math.h>
 #include <stdlib.h>
 
-#include "chunk_image.cuh"
-#include "chunkmap.cuh"
-#include "common.cuh"
+#include "gdn_prep.cuh"
 #include "launch.h"
-#include "tc.cuh"
 #include "tma_host.h"
 
 namespace gdr {
 namespace {
 
 using namespace tc;
-
-constexpr int kC = GDR_CHUNK;
-constexpr int kDK = 128;
-constexpr int kDVS = 32;
-constexpr uint32_t kDrainLimit = 1u << 26;
-
-// The prep's shared-memory staging of P | T | gate factors (e^{G_t}[64],
-// e^{G_last - G_t}[64], e^{G_last}); P and T are copied to the chunk image from here.
-constexpr int WS_T = 16384, WS_G = 32768;
-constexpr size_t kStatusBytes = 256;
-
-// [64][64] fp32 scratch with the column index XOR-ed by the row (conflict-free rows
-// and columns), as in the fused kernel.
-__device__ __forceinline__ int sx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
-
-__device__ __forceinline__ void ld4_sx(const float* base, int k, int klo, int c4, float (&e)[4]) {
-  const float4 f = *reinterpret_cast<const float4*>(base + k * 64 + (c4 ^ (k & 28)));
-  const float v[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-  for (int x = 0; x < 4; ++x) e[x] = v[x ^ klo];
-}
-
-// Strictly lower part of A, stored by 16x16 blocks (a, m), m <= a: block index
-// a(a+1)/2 + m, entry (r, i) at r*16 + (i ^ r).
-__device__ __forceinline__ int pa(int a, int m, int r, int i) {
-  return ((a * (a + 1)) / 2 + m) * 256 + r * 16 + (i ^ r);
-}
-
-__device__ __forceinline__ uint64_t kstep(uint64_t desc0, int rows, int ks) {
-  return desc0 + (uint64_t)((((ks >> 2) * rows * 128) + ((ks & 3) * 32)) >> 4);
-}
-
-__device__ __forceinline__ void st_tile4(unsigned char* tile, int rows, int r, int q, float4 x) {
-  x.x = to_tf32(x.x); x.y = to_tf32(x.y); x.z = to_tf32(x.z); x.w = to_tf32(x.w);
-  *reinterpret_cast<float4*>(tile + swz_off4(r, q, rows)) = x;
-}
-
-// ========================================================================================
-// Kernel 1: per-chunk P, T and gate factors
-// ========================================================================================
-
-constexpr int P_THREADS = 128;
-constexpr int P_QK = 0;                    // bf16 [128][128] SW128 (q rows 0-63, k 64-127)  32 KB
-// once the Gram has been read, the solve's scratch reuses the q/k tile:
-constexpr int P_X = 0;                     //   X scratch, sx() layout                        16 KB
-constexpr int P_A = 16384;                 //   packed strictly-lower A                       10 KB
-constexpr int P_Z = P_A + 10240;           //   level scratch [3][16][16]                      3 KB
-constexpr int P_OUT = 32768;               // P | T | gates (staging)                         33 KB
-constexpr int P_SMALL = P_OUT + 34816;
-constexpr int P_SMEM = P_SMALL + 1024 + 1024;   // 68 KB: three CTAs per SM
-constexpr uint32_t P_TM_COLS = 64;
-
-struct PrepSmall {
-  float g[kC];
-  float beta[kC];
-  uint32_t tmem;
-  unsigned long long tma_bar;
-  unsigned long long mma_bar;
-};
+using namespace gdnprep;
 
 template <unsigned PRO>
-__global__ void __launch_bounds__(P_THREADS)
+__global__ void __launch_bounds__(P_THREADS, 5)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ alpha,
                       const float* __restrict__ beta, unsigned char* __restrict__ ws,
@@ -107,318 +43,22 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + padb;
-  unsigned char* tQK = sm + P_QK;
-  unsigned char* tP = sm + P_OUT;
-  unsigned char* tT = sm + P_OUT + WS_T;
-  float* gates = reinterpret_cast<float*>(sm + P_OUT + WS_G);
-  float* Xs = reinterpret_cast<float*>(sm + P_X);
-  float* As = reinterpret_cast<float*>(sm + P_A);
-  float* Zs = reinterpret_cast<float*>(sm + P_Z);
   PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(&ps.tma_bar);
-  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int gc = blockIdx.x % m.nck;
   const int h = blockIdx.x / m.nck;
-  const ChunkLoc loc = chunk_locate(m, gc);
-  if (!loc.valid) return;            // past the last chunk of the packed sequences
-  const int b = loc.b, t0 = loc.t0, L = loc.L;
-
-  if (tid == 0) {
-    mbar_init(tma_bar, 1);
-    mbar_init(mma_bar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(&ps.tmem, P_TM_COLS);
+  if (!chunk_locate(m, gc).valid) return;   // past the last chunk of the packed sequences
+  if (tid == 0) prep_init(ps);
+  if (tid < 32) tmem_alloc(&ps.tmem, P_TM_COLS);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = ps.tmem;
-  const uint32_t tlane = (uint32_t)(warp * 32) << 16;
-  const uint32_t aQK = smem_u32(tQK);
-  if (tid == 0) {
-    mbar_expect_tx(tma_bar, 32768);
-    tma_load_4d(aQK, &tm_q, 0, h, t0, b, tma_bar);
-    tma_load_4d(aQK + 16384, &tm_q, 64, h, t0, b, tma_bar);
-    tma_load_4d(aQK + 8192, &tm_k, 0, h, t0, b, tma_bar);
-    tma_load_4d(aQK + 16384 + 8192, &tm_k, 64, h, t0, b, tma_bar);
-  }
-  // gates of the chunk (rows past T: alpha 1, beta 0)
-  if (tid < kC) {
-    float a = 1.f, bt = 0.f;
-    if (tid < L) {
-      const long row = ((long)b * m.T + t0 + tid) * H + h;
-      a = alpha[row];
-      bt = beta[row];
-    }
-    ps.g[tid] = tid >= L ? 0.f
-                : (PRO & GDR_PROLOGUE_GATE_LOGIT) ? log_gate_from_logit(a)
-                                                  : log_gate_accurate(a);
-    ps.beta[tid] = bt;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const double g0 = ps.g[2 * lane], g1 = ps.g[2 * lane + 1];
-    double s = g0 + g1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const double n = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += n;
-    }
-    const double ex = s - (g0 + g1);
-    ps.g[2 * lane] = (float)(ex + g0);
-    ps.g[2 * lane + 1] = (float)(ex + g0 + g1);
-  }
-  __syncthreads();
-  if (tid < kC) {
-    const float glast = ps.g[L - 1];
-    gates[tid] = __expf(ps.g[tid]);
-    gates[64 + tid] = __expf(fminf(glast - ps.g[tid], 0.f));
-    if (tid == 0) gates[128] = __expf(glast);
-  }
-  bool failed = false;
-  // ---- Gram [q; k] k^T (bf16 operands are exact) ------------------------------------
-  if (!mbar_wait(tma_bar, 0, spin_limit)) {
-    mbar_wait(tma_bar, 0, kDrainLimit);
-    failed = true;
-  }
-  if (__syncthreads_or(failed)) {
-    if (lane == 0) atomicOr(status, 1u);
-    if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
-    return;
-  }
-  if constexpr ((PRO & GDR_PROLOGUE_L2NORM_QK) != 0) {
-    // row tid of the q/k tile (0-63 q, 64-127 k): divided by its L2 norm in fp32 and
-    // rounded back to bf16, in place, before anything reads it
-    const int r = tid;
-    uint4 x[16];
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      x[i] = *reinterpret_cast<const uint4*>(tQK + (i >> 3) * 16384 + r * 128 +
-                                             (((i & 7) ^ (r & 7)) << 4));
-      const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&x[i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hh[e]);
-        ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
-      }
-    }
-    const float sc = l2_scale(ss);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&x[i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hh[e]);
-        hh[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
-      }
-      *reinterpret_cast<uint4*>(tQK + (i >> 3) * 16384 + r * 128 + (((i & 7) ^ (r & 7)) << 4)) =
-          x[i];
-    }
-    fence_smem_to_async();
-    __syncthreads();
-  }
-  if (warp == 0) {
-    const uint64_t dA = sdesc(aQK, 16, 1024), dB = sdesc(aQK + 8192, 16, 1024);
-    const uint32_t id = idesc_bf16(128, 64);
-#pragma unroll
-    for (int ks = 0; ks < kDK / 16; ++ks)
-      mma_bf16_w(tb, kstep(dA, 128, ks), kstep(dB, 128, ks), id, ks > 0);
-    mma_commit_w(mma_bar);
-  }
-  // ---- while the Gram runs: the carry's images of this chunk (chunk_image.cuh), from the
-  //      q/k tile (which the solve's scratch overwrites later): [Q (.) e^G; K (.) e^G], e^{G_last},
-  //      K^ = (K (.) e^{G_last - G})^T (tokens past L: zero)
-  unsigned char* img = ws + m.img_base + ((size_t)h * m.nck + gc) * img::kChunkWs;
-  {
-    // Each warp store writes four whole 128-byte tile rows: lane l takes 16-byte chunk
-    // l % 8 of row 4 i + l / 8 of a panel (4 tf32 channels, or 4 tokens for K^).
-    const int sub = lane >> 3, cd = lane & 7;
-    // [Q~; K~]: 128 rows x 4 panels of 32 channels
-#pragma unroll 4
-    for (int it = 0; it < 32; ++it) {
-      const int unit = it * 4 + warp;                 // 0..127: (row group, panel)
-      const int pd = unit & 3, r = 4 * (unit >> 2) + sub;
-      const int ch = 32 * pd + 4 * cd;                // first of the 4 channels
-      const uint2 x = *reinterpret_cast<const uint2*>(
-          tQK + (ch >> 6) * 16384 + r * 128 + ((((ch & 63) >> 3) ^ (r & 7)) << 4) + ((ch & 7) << 1));
-      const float eg = gates[r & 63];
-      *reinterpret_cast<float4*>(img + img::WS_QK + pd * 16384 + r * 128 + ((cd ^ (r & 7)) << 4)) =
-          img::tf32x4(__uint_as_float(x.x << 16) * eg, __uint_as_float(x.x & 0xffff0000u) * eg,
-                      __uint_as_float(x.y << 16) * eg, __uint_as_float(x.y & 0xffff0000u) * eg);
-    }
-    reinterpret_cast<float*>(img + img::WS_EGL)[tid] = gates[128];
-    // K^: 128 rows (channels) x 2 panels of 32 tokens; tokens past L are zero
-#pragma unroll 4
-    for (int it = 0; it < 16; ++it) {
-      const int unit = it * 4 + warp;                 // 0..63: (row group, panel)
-      const int pd = unit & 1, c = 4 * (unit >> 1) + sub;
-      float f[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = 32 * pd + 4 * cd + u;
-        const float kv = __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(tQK + swz_off_bf16(64 + j, c, 128)));
-        f[u] = j < L ? kv * gates[64 + j] : 0.f;
-      }
-      *reinterpret_cast<float4*>(img + img::WS_KH + pd * 16384 + c * 128 + ((cd ^ (c & 7)) << 4)) =
-          img::tf32x4(f[0], f[1], f[2], f[3]);
-    }
-  }
-  if (!mbar_wait(mma_bar, 0, spin_limit)) {
-    mbar_wait(mma_bar, 0, kDrainLimit);
-    failed = true;
-  }
-  fence_after_sync();
-  if (__syncthreads_or(failed)) {
-    if (lane == 0) atomicOr(status, 1u);
-    fence_before_sync();
-    if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
-    return;
-  }
-  // ---- P (decayed, lower) to the output image; A (decayed, beta, strictly lower) ------
-  {
-    float d[64], gj[64];
-    tmem_ld32(tb + tlane, *reinterpret_cast<float(*)[32]>(&d[0]));
-    tmem_ld32(tb + tlane + 32, *reinterpret_cast<float(*)[32]>(&d[32]));
-#pragma unroll
-    for (int x = 0; x < 64; ++x) gj[x] = ps.g[x];
-    tmem_wait_ld();
-    const int t = tid & 63;
-    const float gt = ps.g[t];
-    if (tid < 64) {
-#pragma unroll
-      for (int j = 0; j < 64; ++j) d[j] = j <= t ? d[j] * __expf(gt - gj[j]) : 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        st_tile4(tP, 64, t, q, make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]));
-    } else {
-      const float bt = ps.beta[t];
-      const int a = t >> 4, r = t & 15;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const int m = j >> 4;
-        if (m <= a) As[pa(a, m, r, j & 15)] = j < t ? bt * d[j] * __expf(gt - gj[j]) : 0.f;
-      }
-    }
-  }
+  prep_chunk<PRO, 0>(&tm_q, &tm_k, alpha, beta, ws, m, H, gc, h, sm, tb, tid, 0u, status,
+                     spin_limit);
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
-  // ---- X = (I + A)^{-1}: diagonal blocks (one per warp), then three block levels ------------
-  if (lane < 16) {
-    const int a = warp, jl = lane, base = 16 * a;
-    const int bx = base ^ (base & 16);
-    const float* Ab = As + pa(a, a, 0, 0);
-    float x[16];
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) {
-      float a_row[16];
-#pragma unroll
-      for (int i = 0; i < tl; ++i) a_row[i] = Ab[tl * 16 + (i ^ tl)];
-      float acc0 = (tl == jl) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < tl; i += 2) {
-        acc0 = fmaf(-a_row[i], x[i], acc0);
-        if (i + 1 < tl) acc1 = fmaf(-a_row[i + 1], x[i + 1], acc1);
-      }
-      x[tl] = (tl < jl) ? 0.f : acc0 + acc1;
-    }
-    float* Xb = Xs + base * 64 + bx;
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) Xb[tl * 64 + (jl ^ tl)] = x[tl];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int d = 1; d <= 3; ++d) {
-    const int nunits = (4 - d) * 64;           // unit = (block bb, row r, column quad cq)
-    float z[2][4];
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-#pragma unroll
-        for (int m = 0; m < d; ++m)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k = 16 * (bb + m) + i;
-            const float av = As[pa(aa, bb + m, r, i)];
-            float e[4];
-            ld4_sx(Xs, k, i & 3, 16 * bb + 4 * cq, e);
-            z0 = fmaf(av, e[0], z0);
-            z1 = fmaf(av, e[1], z1);
-            z2 = fmaf(av, e[2], z2);
-            z3 = fmaf(av, e[3], z3);
-          }
-        z[n][0] = z0; z[n][1] = z1; z[n][2] = z2; z[n][3] = z3;
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3;
-        *reinterpret_cast<float4*>(&Zs[bb * 256 + r * 16 + 4 * cq]) =
-            make_float4(z[n][0], z[n][1], z[n][2], z[n][3]);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float xa = Xs[sx(16 * aa + r, 16 * aa + i)];
-          const float4 zz = *reinterpret_cast<const float4*>(&Zs[bb * 256 + i * 16 + 4 * cq]);
-          x0 = fmaf(xa, zz.x, x0);
-          x1 = fmaf(xa, zz.y, x1);
-          x2 = fmaf(xa, zz.z, x2);
-          x3 = fmaf(xa, zz.w, x3);
-        }
-        z[n][0] = -x0; z[n][1] = -x1; z[n][2] = -x2; z[n][3] = -x3;
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        const int row = 16 * aa + r, col = 16 * bb + 4 * cq;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Xs[sx(row, col + e)] = z[n][e];
-      }
-    }
-    __syncthreads();
-  }
-  // ---- T = X Diag(beta) (blocks above the diagonal are zero) -------------------------------
-  {
-    const int r = tid & 63, half = tid >> 6;
-    float xr[32];
-#pragma unroll
-    for (int x = 0; x < 32; ++x) {
-      const int j = half * 32 + x;
-      xr[x] = ((j >> 4) <= (r >> 4)) ? Xs[sx(r, j)] * ps.beta[j] : 0.f;
-    }
-#pragma unroll
-    for (int x = 0; x < 8; ++x)
-      st_tile4(tT, 64, r, half * 8 + x,
-               make_float4(xr[4 * x], xr[4 * x + 1], xr[4 * x + 2], xr[4 * x + 3]));
-  }
-  fence_smem_to_async();
-  __syncthreads();
-  if (tid == 0) {
-    bulk_store(img + img::WS_P, smem_u32(tP), 16384);
-    bulk_store(img + img::WS_T, smem_u32(tT), 16384);
-    bulk_commit();
-    bulk_wait_all();
-  }
+  if (tid < 32) tmem_dealloc(tb, P_TM_COLS);
 }
 
 uint32_t split_spin_limit() {
@@ -428,6 +68,12 @@ uint32_t split_spin_limit() {
 }
 
 cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
+  if (gdn_stream_eligible(a, m)) {
+    // few chains: the prep runs alongside the carry in one kernel
+    const cudaError_t e = launch_gdn_stream(a, m, split_spin_limit(), stream);
+    if (e == cudaSuccess) timing_mark(stream, 0);
+    return e;
+  }
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
   CUtensorMap mq, mk;
@@ -454,7 +100,8 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
 
 size_t split_prefill_workspace(int B, int T, int H) {
   const size_t nchunks = ((size_t)T + kC - 1) / kC;
-  return (size_t)B * H * nchunks * img::kChunkWs;
+  // the chunk images, then the streaming prefill's ticket counter and chunk flags
+  return (size_t)B * H * nchunks * img::kChunkWs + gdn_stream_sync_bytes((int)(B * nchunks), H);
 }
 
 size_t split_chunk_image_bytes() { return img::kChunkWs; }
