@@ -251,17 +251,8 @@ class PrefillRunner:
         self.ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev)
         self.path = g.prefill_path(w.dk, w.dv, w.torch_dtype, w.mixer == "kda")
         # the tensor-core path with a full-size workspace runs a per-chunk prep kernel,
-        # then the state carry, or (GDN with at most one chain per SM) both in one
-        # streaming kernel; the others run one kernel per call.  One untimed call,
-        # with the library's per-kernel marks on, tells which.
-        g.timing_start()
-        self.step(0)
-        torch.cuda.synchronize(dev)
-        marks, _ = g.timing_stop()
-        if self.path == "tensor-core" and len(marks) == 1:
-            self.kernels = [f"{w.mixer}_stream_kernel (prep + sliced carry)"]
-            self.kernel_key = f"prefill_stream:{w.name}"
-        elif self.path == "tensor-core":
+        # then the state carry; the others run one kernel per call
+        if self.path == "tensor-core":
             self.kernels = [f"{w.mixer}_chunk_prep_kernel", "state carry (sliced_carry_kernel or row_carry_kernel)"]
             self.kernel_key = f"prefill_two-kernel:{w.name}"
         else:

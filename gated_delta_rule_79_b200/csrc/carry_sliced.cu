@@ -1,5 +1,5 @@
-// The value-sliced state carry kernel of the GDN and KDA two-kernel prefills (its body,
-// carry_sliced.cuh, is shared with the streaming GDN prefill).  It is taken when there are
+// The value-sliced state carry kernel of the GDN and KDA two-kernel prefills (its body is
+// carry_sliced.cuh).  It is taken when there are
 // too few (sequence, head) chains to fill the GPU; otherwise the per-head carry
 // (carry_rows.cu) reads each chunk's operands once instead of once per slice.  NV = 64
 // (two value slices sharing each chunk's operands) is taken when that still gives every
@@ -35,8 +35,8 @@ sliced_carry_kernel(const __grid_constant__ CUtensorMap tm_v,
   __syncthreads();
   fence_after_sync();
   const uint32_t tb = cs.tmem;
-  carry_body<NV, Tout, false>(&tm_v, ws, s0, o, s_final, m, H, dv, status, spin_limit,
-                              (int)blockIdx.x, sm, tb, tid, nullptr);
+  carry_body<NV, Tout>(&tm_v, ws, s0, o, s_final, m, H, dv, status, spin_limit,
+                       (int)blockIdx.x, sm, tb, tid);
   fence_before_sync();
   __syncthreads();
   if (tid < 32) tmem_dealloc(tb, Lay::COLS);

@@ -20,9 +20,7 @@
 // operand tile.
 //
 // carry_body is the whole of one carry CTA after its barriers are initialised and its
-// tensor memory allocated; it runs in the stand-alone carry kernel (carry_sliced.cu),
-// which follows a prep kernel, and in the streaming GDN prefill (prefill_stream.cu),
-// where it reads each chunk's image as soon as a prep group on some SM has published it.
+// tensor memory allocated (the kernel is carry_sliced.cu).
 //
 // Precision: kind::tf32 products with operands rounded to nearest.  Waits are bounded; a
 // give-up records GDR_ERR_TIMEOUT in the workspace status word, drains what was issued
@@ -103,27 +101,16 @@ __device__ __forceinline__ void carry_init(CarrySmall& cs) {
   fence_mbar_init();
 }
 
-// Polls a publication flag (acquire, GPU scope) until it is set; false after `limit`
-// polls.
-__device__ __forceinline__ bool wait_ready(const unsigned* flag, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (ld_acquire_gpu(flag) != 0u) return true;
-    __nanosleep(64);
-  }
-  return false;
-}
-
 // One carry CTA: chain `chain` = (sequence, head, slice) in slice-fastest order, threads
 // tid = 0..255 of the CTA, shared memory `sm` (1024-aligned, CarryLayout<NV>), tensor
-// memory columns [tb, tb + CarryLayout<NV>::COLS).  With STREAM, chunk gc of head h is
-// read once ready_flags[h * m.nck + gc] is set.
-template <int NV, typename Tout, bool STREAM>
+// memory columns [tb, tb + CarryLayout<NV>::COLS).
+template <int NV, typename Tout>
 __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsigned char* ws,
                                            const float* s0, Tout* o, float* s_final,
                                            const ChunkMap& m, int H, int dv,
                                            unsigned int* status, uint32_t spin_limit,
-                                           int chain, unsigned char* sm, uint32_t tb, int tid,
-                                           const unsigned* ready_flags) {
+                                           int chain, unsigned char* sm, uint32_t tb,
+                                           int tid) {
   using Lay = CarryLayout<NV>;
   constexpr int NB = NV / 32;        // blocks of 32 value columns
   CarrySmall& cs = *reinterpret_cast<CarrySmall*>(sm + Lay::SMALL);
@@ -213,17 +200,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
         const uint32_t bytes[NG] = {WS_A_BYTES, 16384, WS_D_BYTES};
         last_par = par;
         pending = 0;
-        bool ready = true;
-        if constexpr (STREAM) {
-          // the chunk's image is read only once the prep has published it
-          ready = wait_ready(ready_flags + (size_t)h * m.nck + first + c, spin_limit);
-          if (!ready) {
-            atomicOr(status, 1u);
-            cs.abort = 1;
-          }
-          fence_global_to_async();
-        }
-        for (int g = 0; g < NG && ready; ++g) {
+        for (int g = 0; g < NG; ++g) {
           if (!mbar_wait(empty + g, par ^ 1u, spin_limit)) {
             give_up(empty + g, par ^ 1u, false);
             break;
@@ -239,7 +216,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
           }
           pending |= 1u << g;
         }
-        if (!STREAM && c + 1 < nchunks) bulk_prefetch_l2(src + kChunkWs, kChunkWs);
+        if (c + 1 < nchunks) bulk_prefetch_l2(src + kChunkWs, kChunkWs);
       }
       named_bar(2, 128);
       if (cs.abort) break;

@@ -14,9 +14,8 @@
 // CUDA cores by 16 x 16 blocks.  The image holds [Q (.) e^G; K (.) e^G], e^{G_last}, T,
 // (K (.) e^{G_last - G})^T and P as tf32 tiles.
 //
-// prep_chunk is the work of one 128-thread group for one chunk; it runs in the
-// stand-alone prep kernel (prefill_split.cu, one chunk per CTA) and in the prep warps of
-// the streaming GDN prefill (prefill_stream.cu, chunk after chunk).
+// prep_chunk is the work of one 128-thread group for one chunk (the kernel is
+// prefill_split.cu, one chunk per CTA); a group may run it for chunk after chunk.
 #pragma once
 
 #include <cuda.h>

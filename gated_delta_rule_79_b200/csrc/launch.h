@@ -62,16 +62,6 @@ size_t kda_split_workspace(int B, int T, int H);
 size_t split_chunk_image_bytes();
 size_t kda_chunk_image_bytes();
 cudaError_t launch_prefill_split(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream);
-
-// prefill_stream.cu: the streaming GDN prefill (prep and sliced carry in one persistent
-// kernel) for a dense batch with at most one (sequence, head, 32-column slice) chain per
-// SM.  Its ticket counter and per-chunk flags follow the chunk images in the workspace
-// (gdn_stream_sync_offset, gdn_stream_sync_bytes).
-size_t gdn_stream_sync_bytes(int nck, int H);
-size_t gdn_stream_sync_offset(const ChunkMap& m, int H);
-bool gdn_stream_eligible(const PrefillArgs& a, const ChunkMap& m);
-cudaError_t launch_gdn_stream(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
-                              cudaStream_t stream);
 cudaError_t launch_prefill_kda_split(const PrefillArgs& a, const ChunkMap& m,
                                      cudaStream_t stream);
 // The state carry both two-kernel prefills share, run after the prep kernel has written

@@ -68,12 +68,6 @@ uint32_t split_spin_limit() {
 }
 
 cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
-  if (gdn_stream_eligible(a, m)) {
-    // few chains: the prep runs alongside the carry in one kernel
-    const cudaError_t e = launch_gdn_stream(a, m, split_spin_limit(), stream);
-    if (e == cudaSuccess) timing_mark(stream, 0);
-    return e;
-  }
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
   CUtensorMap mq, mk;
@@ -100,8 +94,7 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
 
 size_t split_prefill_workspace(int B, int T, int H) {
   const size_t nchunks = ((size_t)T + kC - 1) / kC;
-  // the chunk images, then the streaming prefill's ticket counter and chunk flags
-  return (size_t)B * H * nchunks * img::kChunkWs + gdn_stream_sync_bytes((int)(B * nchunks), H);
+  return (size_t)B * H * nchunks * img::kChunkWs;
 }
 
 size_t split_chunk_image_bytes() { return img::kChunkWs; }

@@ -257,62 +257,41 @@ def test_many_chains_take_the_per_head_carry():
     check(o[picks], s[picks], o_ref, s_ref, TOL["bf16"], "many chains")
 
 
-def _kernels_per_call(run):
-    """How many kernels one prefill call launched (the library's timing marks)."""
-    import gated_delta_rule_79_b200 as g
-    g.timing_start()
-    run()
-    torch.cuda.synchronize()
-    ms, calls = g.timing_stop()
-    assert calls == 1
-    return len(ms)
 
-
-@pytest.mark.parametrize("stream", ["1", "0"])
 @pytest.mark.parametrize("B,H,T,dv", [(1, 4, 200, 128), (2, 3, 129, 64), (1, 1, 64, 32),
                                       (1, 37, 130, 128), (3, 1, 1000, 128)])
 @pytest.mark.parametrize("init", [True, False])
-def test_gdn_streaming_prefill(stream, B, H, T, dv, init, monkeypatch):
-    """GDN with few (sequence, head, 32-column slice) chains runs the prep and the carry
-    in one persistent kernel (GDR_STREAM=0 keeps the two-kernel prefill): ragged tails,
-    one chunk, exactly as many chains as 148 SMs can hold, long chains, with and without
-    an entering state."""
-    monkeypatch.setenv("GDR_STREAM", stream)
-    w = Workload("stream", "gdn", B, H, T, 128, dv, "bf16", "randn")
+def test_gdn_prefill_chain_counts(B, H, T, dv, init):
+    """GDN on the value-sliced carry: ragged tails, one chunk, exactly as many
+    (sequence, head, 32-column slice) chains as 148 SMs hold, long chains, with and
+    without an entering state."""
+    w = Workload("chains", "gdn", B, H, T, 128, dv, "bf16", "randn")
     x = make_inputs(w, seed=B * 100 + H + T, gates="slow")
     if not init:
         x["s0"] = None
-    import gated_delta_rule_79_b200 as g
-    t = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
-    out = {}
-
-    def run():
-        out["o"], out["s"] = g.gdn_prefill(t["q"], t["k"], t["v"], t["alpha"], t["beta"], t["s0"],
-                                           out_dtype=torch.float32)
-    n = _kernels_per_call(run)
-    chains = B * H * dv // 32
-    assert n == (1 if stream == "1" and chains <= torch.cuda.get_device_properties(0).multi_processor_count else 2)
+    o, s = gpu_prefill("gdn", x, out_dtype=torch.float32)
     o_ref, s_ref = ref_prefill(x)
-    check(to_np(out["o"]), to_np(out["s"]), o_ref, s_ref, TOL["bf16"],
-          f"stream={stream} B={B} H={H} T={T} dv={dv}")
+    check(o, s, o_ref, s_ref, TOL["bf16"], f"B={B} H={H} T={T} dv={dv}")
 
 
-def test_gdn_streaming_prefill_bf16_out_repeated():
+@pytest.mark.parametrize("mixer", ["gdn", "kda"])
+def test_prefill_bf16_out_repeated(mixer):
     """bf16 outputs, the final state over the entering one, and the same workspace for
-    several calls in a row (the chunk flags are cleared before each)."""
+    several calls in a row."""
     import gated_delta_rule_79_b200 as g
-    w = Workload("stream16", "gdn", 1, 8, 300, 128, 128, "bf16", "randn")
+    w = Workload("rep16", mixer, 1, 8, 300, 128, 128, "bf16", "randn")
     x = make_inputs(w, seed=5, gates="slow")
     t = {k: v.cuda() for k, v in x.items()}
-    ws, _ = g.prefill_workspace(1, 300, 8, 128, 128, False, torch.device("cuda"))
+    fn = g.kda_prefill if mixer == "kda" else g.gdn_prefill
+    ws, _ = g.prefill_workspace(1, 300, 8, 128, 128, mixer == "kda", torch.device("cuda"))
     s_ref = x["s0"].double().numpy()
     state = t["s0"].clone()
     for it in range(3):
-        o, _ = g.gdn_prefill(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state,
-                             workspace=ws)
+        o, _ = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state,
+                  workspace=ws)
         torch.cuda.synchronize()
         g.workspace_status(ws)
         args = [x[k].double().numpy() for k in ("q", "k", "v", "alpha", "beta")]
         o_ref, s_ref = gated_delta_rule(*args, s_ref)
-        check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"stream bf16 call {it}")
+        check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{mixer} bf16 call {it}")
         s_ref = to_np(state).astype(np.float64)
