@@ -273,8 +273,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
       if (!mbar_wait(mma_bar, mphase, spin_limit)) give_up(mma_bar, mphase, true);
       mphase ^= 1u;
       fence_after_sync();
-      named_bar(1, R_CARRY);
-      return cs.abort != 0;
+      return named_bar_or(1, R_CARRY, cs.abort != 0);
     };
     // S <- x (.) e^{G_last} (the decay of the chunk whose [Q~; K~] | e^{G_last} copy is in
     // shared memory) and the operand copy <- tf32(x), one block of 32 channels
@@ -350,8 +349,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
     // ---- the entering state (rows past d_v zero), decayed by the first chunk's gates -------
     // (a full barrier's copies are the loader's to drain, the products' are this group's)
     if (nchunks > 0 && !mbar_wait(full + G_A, 0, spin_limit)) give_up(full + G_A, 0, false);
-    named_bar(1, R_CARRY);
-    aborted = cs.abort != 0;
+    aborted = named_bar_or(1, R_CARRY, cs.abort != 0);
     if (!aborted) {
 #pragma unroll
       for (int nh = 0; nh < 2; ++nh) {
@@ -371,13 +369,13 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
       tmem_wait_st();
     }
     fence_before_sync();
-    named_bar(1, R_CARRY);
+    aborted = named_bar_or(1, R_CARRY, cs.abort != 0) || aborted;
     for (int c = 0; c < nchunks && !aborted; ++c) {
       const uint32_t pc = (uint32_t)c & 1u;
       const uint32_t tD = T_D + 128u * pc;
       // [Q~; K~] has landed (waited for before the decay); this D buffer was read when the
-      // outputs of chunk c - 2 were staged
-      if ((aborted = cs.abort != 0)) break;
+      // outputs of chunk c - 2 were staged (a give-up anywhere stops the loop at the barrier
+      // that ends the previous chunk)
       fence_after_sync();
       // ---- Y^T = S0 K~^T (the loader issues O1^T = S0 Q~^T behind it) -----------------------
       if (warp == 0) {
@@ -464,7 +462,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
       tmem_wait_st();
       if (tid == R_STORER) bulk_wait_read_all();   // the staging tile is free for the next chunk
       fence_before_sync();
-      named_bar(1, R_CARRY);
+      aborted = named_bar_or(1, R_CARRY, cs.abort != 0);
     }
     if (!aborted && nchunks > 0) {
       stage_outputs(nchunks - 1);

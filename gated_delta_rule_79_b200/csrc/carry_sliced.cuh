@@ -147,8 +147,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
       const uint32_t use = (uint32_t)(cc >> 1);
       uint64_t* ofull = reinterpret_cast<uint64_t*>(&cs.out_full[ob]);
       if (lt == 0 && !mbar_wait(ofull, use & 1u, spin_limit)) give_up(ofull, use & 1u, false);
-      named_bar(2, 128);
-      if (cs.abort) return false;
+      if (named_bar_or(2, 128, cs.abort != 0)) return false;
       fence_after_sync();
       const ChunkLoc loc = chunk_locate(m, first + cc);
       const int t = 32 * q4 + lane;
@@ -218,16 +217,17 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
         }
         if (c + 1 < nchunks) bulk_prefetch_l2(src + kChunkWs, kChunkWs);
       }
-      named_bar(2, 128);
-      if (cs.abort) break;
+      if (named_bar_or(2, 128, cs.abort != 0)) break;
       if (c > 0 && !write_outputs(c - 1)) break;
     }
-    if (cs.abort && lt == 0) {
+    // one decision for the whole warpgroup (a give-up elsewhere may land between reads)
+    const bool ab = named_bar_or(2, 128, cs.abort != 0);
+    if (ab && lt == 0) {
       // copies this thread issued may still be landing in shared memory: let them finish
       for (int g = 0; g < NG; ++g)
         if (pending & (1u << g)) mbar_wait(full + g, last_par, kDrainLimit);
     }
-    if (!cs.abort && nchunks > 0) write_outputs(nchunks - 1);
+    if (!ab && nchunks > 0) write_outputs(nchunks - 1);
   } else {
     // =========================== carry warpgroup ======================================
     const long sbase = ((long)chunk_state_index(m, seq) * H + h) * (long)dv * kDK;
@@ -254,8 +254,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
       if (!mbar_wait(mma_bar, mphase, spin_limit)) give_up(mma_bar, mphase, true);
       mphase ^= 1u;
       fence_after_sync();
-      named_bar(1, 128);
-      return cs.abort != 0;
+      return named_bar_or(1, 128, cs.abort != 0);
     };
     bool aborted = false;
     for (int c = 0; c < nchunks; ++c) {
@@ -270,8 +269,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
           if (!mbar_wait(oe, p2, spin_limit)) give_up(oe, p2, false);
         }
       }
-      named_bar(1, 128);
-      if ((aborted = cs.abort != 0)) break;
+      if ((aborted = named_bar_or(1, 128, cs.abort != 0))) break;
       fence_after_sync();
       // ---- decay the state in TMEM, then [O1; Y] = [Q~; K~] S0^T -----------------------------
       {
