@@ -13,8 +13,9 @@
 // The per-token update is the decode step (decode.cu): for row r of S,
 //     s~ = S[r,:] (.) alpha_t;  a = s~ . k_t;  b = s~ . q_t;  u = beta_t (v_t[r] - a)
 //     S[r,:] = s~ + u k_t;      o_t[r] = b + u (k_t . q_t)
-// Layout: one warp per (sequence, head), a state row spread over 8 lanes in float4
-// pieces; each row group is read from HBM once, carried through the K tokens in
+// Layout: two warps per (sequence, head), each over half of the rows (more, shorter
+// tasks: the last partial wave of the grid is a smaller share), a state row spread over
+// 8 lanes in float4 pieces; each row group is read from HBM once, carried through the K tokens in
 // registers, and each snapshot row is written once (evict-first).  The K tokens' q, k
 // and gates, and k_t . q_t, are staged in shared memory per warp.  Bound: HBM, with
 // (1 + K) d_v d_k 4 bytes per (sequence, head) (2 d_v d_k 4 without snapshots).
@@ -42,9 +43,13 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 
   extern __shared__ float vsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long head = (long)blockIdx.x * kWarps + warp;   // n * H + h
+  // two warps per (sequence, head), each over half of the d_v rows
+  const long task = (long)blockIdx.x * kWarps + warp;
   const long NH = (long)N * H;
-  if (head >= NH) return;
+  if (task >= 2 * NH) return;
+  const long head = task >> 1;                          // n * H + h
+  const int rows = dv >> 1;
+  const int rbase = (int)(task & 1) * rows;
   const long n = head / H, h = head % H;
   // per warp: K x (q[DK], k[DK], gate[GA], {beta, k.q, -, -})
   const int per_tok = 2 * DK + GA + 4;
@@ -91,10 +96,14 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 
   const int sub = lane / LPR;
   const int j = lane % LPR;
-  float* Sh = state + head * (long)dv * DK;
+  // this warp's rows, as if they were the whole state
+  float* Sh = state + (head * (long)dv + rbase) * DK;
   const long snap_stride = NH * (long)dv * DK;       // one snapshot = one full state
+  float* Snb = snaps ? snaps + (head * (long)dv + rbase) * DK : nullptr;
+  const Tin* vb = v + rbase;
+  Tout* obase = o + rbase;
 
-  for (int r0 = 0; r0 < dv; r0 += RPW * ITER) {
+  for (int r0 = 0; r0 < rows; r0 += RPW * ITER) {
     float4 s[ITER][F4];
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
@@ -118,7 +127,7 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
       const float bt = tk[2 * DK + GA], kq = tk[2 * DK + GA + 1];
       float vr[ITER];
 #pragma unroll
-      for (int it = 0; it < ITER; ++it) vr[it] = Elem<Tin>::load(v + trow * dv + r0 + it * RPW + sub);
+      for (int it = 0; it < ITER; ++it) vr[it] = Elem<Tin>::load(vb + trow * dv + r0 + it * RPW + sub);
 #pragma unroll
       for (int it = 0; it < ITER; ++it) {
         const int row = r0 + it * RPW + sub;
@@ -149,11 +158,11 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 #pragma unroll
           for (int x = 0; x < 4; ++x) e[x] = fmaf(u, kk[x], e[x]);
           if (snaps)
-            __stcs(reinterpret_cast<float4*>(snaps + t * snap_stride + head * (long)dv * DK +
-                                             (long)row * DK + 4 * (j + LPR * m)),
+            __stcs(reinterpret_cast<float4*>(Snb + t * snap_stride + (long)row * DK +
+                                             4 * (j + LPR * m)),
                    s[it][m]);
         }
-        if (j == 0) Elem<Tout>::store(o + trow * dv + row, fmaf(u, kq, pb));
+        if (j == 0) Elem<Tout>::store(obase + trow * dv + row, fmaf(u, kq, pb));
       }
     }
     if (!snaps) {
@@ -171,7 +180,7 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 template <int DK, bool KDA, typename Tin>
 cudaError_t launch_t(const VerifyArgs& a, cudaStream_t st) {
   const long NH = (long)a.N * a.H;
-  const int grid = (int)((NH + kWarps - 1) / kWarps);
+  const int grid = (int)((2 * NH + kWarps - 1) / kWarps);
   constexpr int GA = KDA ? DK : 4;
   const size_t smem = (size_t)kWarps * a.K * (2 * DK + GA + 4) * sizeof(float);
   cudaError_t e;
