@@ -34,6 +34,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -189,7 +190,9 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples (one CSV per rank); GDR_CLOCKS_DIR keeps them somewhere chosen
+        self.path = os.path.join(os.environ.get("GDR_CLOCKS_DIR") or tempfile.gettempdir(),
+                                 f"gdr_clocks_rank{index}.csv")
 
     def start(self):
         try:
