@@ -80,3 +80,22 @@ def test_verify_algorithmic_bytes_count_state_and_snapshots():
     nb, flops = bench.algorithmic(w)
     assert (1 + w.T) * state < nb < (1 + w.T) * state * 1.02
     assert flops == w.B * w.T * w.H * 6 * w.dk * w.dv
+
+
+def test_traffic_records_name_their_sources_and_captures():
+    """Every DRAM-traffic record in profiles/traffic.json names source files that exist
+    and the committed summary it came from; a record is used only while the digest of
+    those sources is unchanged."""
+    import json
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    recs = json.load(open(os.path.join(root, "profiles", "traffic.json")))
+    assert recs
+    for key, rec in recs.items():
+        srcs = rec["source"] if isinstance(rec["source"], list) else [rec["source"]]
+        for src in srcs:
+            assert os.path.exists(os.path.join(root, src)), (key, src)
+        assert os.path.exists(os.path.join(root, rec["capture"])), key
+        assert rec["dram_bytes_per_launch"] > 0
+        current = bench.source_sha(rec["source"]) == rec["source_sha"]
+        assert (bench.load_traffic(key) is not None) == current, key
+    assert bench.load_traffic("no such kernel") is None
