@@ -102,3 +102,76 @@ def test_public_names_resolve():
     import gated_delta_rule_79_b200 as g
     for name in g.__all__:
         assert getattr(g, name) is not None, name
+
+
+@pytest.mark.parametrize("fn", ["gdn_verify", "kda_verify"])
+def test_verify_rejects_bad_arguments(g, fn):
+    f, fx = getattr(g.lib, fn), getattr(g.lib, fn + "_ex")
+    P = 1 << 20
+
+    def call(ex=None, **kw):
+        a = dict(q=P, k=P, v=P, alpha=P, beta=P, state=P, snaps=P, o=P, N=4, K=3, H=2,
+                 dk=128, dv=64, i=1, oo=1)
+        a.update(kw)
+        args = (a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["state"], a["snaps"], a["o"],
+                a["N"], a["K"], a["H"], a["dk"], a["dv"], a["i"], a["oo"], None)
+        return f(*args) if ex is None else fx(*args, ex)
+    assert call(K=0) == g.GDR_ERR_UNSUPPORTED
+    assert call(K=17) == g.GDR_ERR_UNSUPPORTED
+    assert call(dk=48) == g.GDR_ERR_UNSUPPORTED
+    assert call(N=-1) == g.GDR_ERR_INVALID_ARG
+    assert call(state=None) == g.GDR_ERR_INVALID_ARG
+    assert call(snaps=P + 4) == g.GDR_ERR_INVALID_ARG
+    assert call(oo=3) == g.GDR_ERR_INVALID_ARG
+    assert call(ex=4) == g.GDR_ERR_INVALID_ARG
+    assert "prologue" in g.lib.gdr_last_error().decode()
+    assert call(N=0) == g.GDR_OK
+
+
+@pytest.mark.parametrize("fn", ["gdn_prefill_varlen", "kda_prefill_varlen"])
+def test_varlen_rejects_bad_arguments(g, fn):
+    f, fx = getattr(g.lib, fn), getattr(g.lib, fn + "_ex")
+    P = 1 << 20
+
+    def call(ex=None, **kw):
+        a = dict(q=P, k=P, v=P, alpha=P, beta=P, cu=P, slots=None, state=P, o=P, nseq=3,
+                 total=100, H=2, dk=128, dv=128, i=g.GDR_BF16, oo=1, chunk=64, ws=P,
+                 nws=1 << 30)
+        a.update(kw)
+        args = (a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["cu"], a["slots"], a["state"],
+                a["o"], a["nseq"], a["total"], a["H"], a["dk"], a["dv"], a["i"], a["oo"],
+                a["chunk"], a["ws"], a["nws"], None)
+        return f(*args) if ex is None else fx(*args, ex)
+    assert call(chunk=32) == g.GDR_ERR_UNSUPPORTED
+    assert call(dk=64) == g.GDR_ERR_UNSUPPORTED
+    assert call(i=g.GDR_F32) == g.GDR_ERR_UNSUPPORTED
+    assert call(nseq=-1) == g.GDR_ERR_INVALID_ARG
+    assert call(cu=None) == g.GDR_ERR_INVALID_ARG
+    assert call(cu=P + 2) == g.GDR_ERR_INVALID_ARG
+    assert call(ws=None) == g.GDR_ERR_INVALID_ARG
+    assert call(nws=256) == g.GDR_ERR_INVALID_ARG
+    assert call(ex=8) == g.GDR_ERR_INVALID_ARG
+    assert call(nseq=0) == g.GDR_OK
+
+
+@pytest.mark.parametrize("fn", ["gdn_backward", "kda_backward"])
+def test_backward_rejects_bad_arguments(g, fn):
+    f = getattr(g.lib, fn)
+    P = 1 << 20
+
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, alpha=P, beta=P, s0=None, dO=P, dsf=None, dq=P, dk_out=P,
+                 dv_out=P, dalpha=P, dbeta=P, ds0=P, B=2, T=100, H=2, dk=128, dv=128,
+                 i=1, do=1, ws=P, nws=1 << 30)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["s0"], a["dO"], a["dsf"],
+                 a["dq"], a["dk_out"], a["dv_out"], a["dalpha"], a["dbeta"], a["ds0"], a["B"],
+                 a["T"], a["H"], a["dk"], a["dv"], a["i"], a["do"], a["ws"], a["nws"], None)
+    assert call(dk=48) == g.GDR_ERR_UNSUPPORTED
+    assert call(B=-1) == g.GDR_ERR_INVALID_ARG
+    assert call(i=7) == g.GDR_ERR_INVALID_ARG
+    assert call(dq=None) == g.GDR_ERR_INVALID_ARG
+    assert call(ds0=None) == g.GDR_ERR_INVALID_ARG
+    assert call(dO=P + 8) == g.GDR_ERR_INVALID_ARG
+    assert call(ws=None) == g.GDR_ERR_INVALID_ARG
+    assert call(B=0) == g.GDR_OK
