@@ -2,6 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+With no --workload the line's top level is gdn_prefill and its "workloads" object
+holds kda_prefill, decode_gdn, decode_kda and kda_long, each timed in the same run
+with its own steps, roofline, clocks, end-to-end figure and oracle baseline.
+
 Workloads (synthetic inputs, recipe in synth/):
   gdn_prefill  GDN chunked prefill, B=1 H=32 T=4096 d=128 bf16       (default)
   kda_prefill  KDA chunked prefill, same shapes, per-channel gates
@@ -626,11 +630,19 @@ class OracleTimer:
         self.sample = (f"{self.cores} processes x {what} of {w.name} per pass, fp64 numpy "
                        f"oracle, one spawn process per core; tokens/s = token-heads/s / H")
 
+    def tokens_per_pass(self):
+        """Tokens (token-heads / H) one sampled pass processes."""
+        return self.cores * self.t_sample * self.tokens_per_unit / self.w.H
+
     def rate(self):
+        return self.timed_pass()[0]
+
+    def timed_pass(self):
+        """One sampled pass: (tokens/s, wall seconds)."""
         t0 = time.perf_counter()
         self.pool.map(_oracle_slice, self.chains)
         wall = time.perf_counter() - t0
-        return self.cores * self.t_sample * self.tokens_per_unit / wall / self.w.H
+        return self.tokens_per_pass() / wall, wall
 
     def close(self):
         self.pool.close()
@@ -639,53 +651,45 @@ class OracleTimer:
 
 # ----------------------------------------------------------------------------------------
 
-def main():
-    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None)
-    ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", default="gdn_prefill", choices=sorted(WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    a = ap.parse_args()
-    w = WORKLOADS[a.workload]
-    if w.name == "gdn_seq_f32":
-        raise SystemExit("gdn_seq_f32 is a parity case, not a bench line")
-    default_steps = 5 if (w.decode or w.name == "kda_long") else 20 if w.verify else 50
-    steps = a.steps if a.steps is not None else default_steps
-    warmup = max(3, a.warmup if a.warmup is not None else 5)
-    rank, world, local = dist_env()
+DEFAULT_WORKLOAD = "gdn_prefill"
+# The other configurations the default run times (each with its own roofline, clocks and
+# end-to-end figure), so that one invocation covers every bf16 configuration of the path.
+DEFAULT_EXTRA = ("kda_prefill", "decode_gdn", "decode_kda", "kda_long")
 
-    if a.impl == "reference":
-        if rank != 0:
-            return 0
-        ot = OracleTimer(w, budget_s=min(10.0, 150.0 / max(1, steps + warmup)))
-        for _ in range(warmup):
-            ot.rate()
-        rates = [ot.rate() for _ in range(steps)]
-        ot.close()
-        v = statistics.median(rates)
-        cores, sample = ot.cores, ot.sample
-        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": a.gpus,
-                "steps": steps, "warmup": warmup, "ms_per_step": tokens(w) / v * 1e3,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
-                           "dv": w.dv, "in_dtype": w.dtype},
-                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores,
-                                 "kind": "oracle", "sample": sample},
-                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        return 0
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    active = dist_init(world, "nccl")
-    peaks, peak_kind = load_peaks()
+def default_steps(w):
+    return 5 if (w.decode or w.name == "kda_long") else 20 if w.verify else 50
+
+
+def run_reference(w, steps, warmup, n_gpus):
+    """The reference arm: the fp64 oracle on the host cores.  One step is one bounded
+    sample pass of the workload (a fixed number of whole (batch, head) chains over a
+    token prefix), timed by the wall clock; ms_per_step is that pass's measured time."""
+    ot = OracleTimer(w, budget_s=min(10.0, 120.0 / max(1, steps + warmup)))
+    for _ in range(warmup):
+        ot.timed_pass()
+    passes = [ot.timed_pass() for _ in range(steps)]
+    ot.close()
+    v = statistics.median(r for r, _ in passes)
+    wall_ms = statistics.median(t for _, t in passes) * 1e3
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": n_gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": wall_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "step": "one bounded sample pass of the workload on the host cores (not a whole "
+                    "call): ms_per_step is its measured wall time",
+            "tokens_per_step": ot.tokens_per_pass(),
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+                       "dv": w.dv, "in_dtype": w.dtype},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": ot.cores,
+                             "kind": "oracle", "sample": ot.sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def run_ours(w, steps, warmup, dev, rank, world, active, peaks, peak_kind, e2e=True,
+             cpu_budget=12.0):
+    """Time workload w on this rank's GPU; returns its JSON record (rank 0's view)."""
     runner = (DecodeRunner if w.decode else VerifyRunner if w.verify
               else VarlenRunner if w.varlen else BackwardRunner if w.backward
               else PrefillRunner)(w, dev, seed=1000 * rank)
@@ -693,7 +697,6 @@ def main():
     clocks.start()
     total_ms, per, kernel_ms = time_device(runner, steps, warmup, dev, active)
     clk = clocks.stop()
-    ms_step = total_ms / steps
     max_ms = max_over_ranks(total_ms, active, dev)
     ntok = tokens(w)
     value = aggregate(ntok * steps, max_ms, world)
@@ -756,22 +759,78 @@ def main():
             "roofline": roofline, **extra,
             "gpu_launches": runner.launches_per_step * steps,
             "clocks": clk}
-    if not a.no_e2e:
-        line["e2e"] = time_e2e(w, dev, steps=max(1, min(steps, 10)), warmup=2, seed=rank)
+    del runner
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if e2e:
+        big = w.name == "kda_long"
+        line["e2e"] = time_e2e(w, dev, steps=max(1, min(steps, 3 if big else 10)),
+                               warmup=1 if big else 2, seed=rank)
         if world > 1:
             line["e2e"]["value"] *= world
-    if rank == 0 and not a.no_cpu_baseline and world == 1:
-        ot = OracleTimer(w, budget_s=12.0)
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    if rank == 0 and cpu_budget and world == 1:
+        ot = OracleTimer(w, budget_s=cpu_budget)
         rate = ot.rate()
         ot.close()
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": ot.cores,
                                 "kind": "oracle", "sample": ot.sample}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help=f"one workload alone (default: {DEFAULT_WORKLOAD}, with "
+                         f"{', '.join(DEFAULT_EXTRA)} under 'workloads')")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    w = WORKLOADS[a.workload or DEFAULT_WORKLOAD]
+    if w.name == "gdn_seq_f32":
+        raise SystemExit("gdn_seq_f32 is a parity case, not a bench line")
+    steps = a.steps if a.steps is not None else default_steps(w)
+    warmup = max(3, a.warmup if a.warmup is not None else 5)
+    rank, world, local = dist_env()
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(w, steps, warmup, a.gpus)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    active = dist_init(world, "nccl")
+    peaks, peak_kind = load_peaks()
+    cpu = None if a.no_cpu_baseline else 12.0
+    line = run_ours(w, steps, warmup, dev, rank, world, active, peaks, peak_kind,
+                    e2e=not a.no_e2e, cpu_budget=cpu)
+    if a.workload is None:
+        # the other configurations, each on its own clock record
+        subs = {}
+        for name in DEFAULT_EXTRA:
+            wx = WORKLOADS[name]
+            sx = a.steps if a.steps is not None else default_steps(wx)
+            sub = run_ours(wx, sx, warmup, dev, rank, world, active, peaks, peak_kind,
+                           e2e=not a.no_e2e, cpu_budget=None if cpu is None else 5.0)
+            for key in ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline",
+                        "data"):
+                sub.pop(key, None)
+            subs[name] = sub
+        line["workloads"] = subs
     if rank == 0:
         print(json.dumps(line), flush=True)
     if active:
         import torch.distributed as dist
         dist.destroy_process_group()
-    del ms_step
     return 0
 
 

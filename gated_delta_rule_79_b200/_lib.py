@@ -22,7 +22,7 @@ CHUNK = 64
 
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
-           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_timing_start", "gdr_timing_stop",
+           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_noalloc_status", "gdr_timing_start", "gdr_timing_stop",
            "gdn_verify", "kda_verify", "gdr_prefill_varlen_workspace_bytes",
            "gdn_prefill_varlen", "kda_prefill_varlen", "gdr_backward_workspace_bytes",
            "gdn_backward", "kda_backward", "gdn_prefill_ex", "kda_prefill_ex", "gdn_decode_ex",
@@ -85,6 +85,8 @@ def _load():
                       i, i, i, i, i, i, i, vp, sz, vp]
     lib.gdn_prefill_noalloc.restype = i
     lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
+    lib.gdr_noalloc_status.restype = i
+    lib.gdr_noalloc_status.argtypes = [vp]
     lib.gdr_prefill_path.restype = i
     lib.gdr_prefill_path.argtypes = [i, i, i, i]
     lib.gdr_workspace_status.restype = i

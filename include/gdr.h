@@ -194,20 +194,30 @@ GDR_API gdr_status kda_decode(const void* q, const void* k, const void* v,
  * and embedders whose device memory is owned by another allocator under a fixed
  * budget.  Arguments, results and errors are those of gdn_prefill without the
  * workspace: the library uses a static device array of 4096 bytes instead,
- * reserved on every GPU that loads the library until the process exits, which
- * runs the single-kernel prefill (it needs the 256-byte status word only).
- * Sizes that would need more scratch are rejected with GDR_ERR_INVALID_ARG.  The
- * first call on a device looks up the array's device address with the device
- * current, so make that first call before any stream capture.  The call
- * allocates nothing and clears the array's status word after launching, so
- * device-side timeouts of this variant are not reported (use gdn_prefill with a
- * workspace and gdr_workspace_status for that).  All calls share the one array:
- * calls that overlap on the GPU (streams without ordering between them) race. */
+ * reserved on every GPU that loads the library until the process exits.  The
+ * prefill it runs (the single-kernel tensor-core kernel for bf16 inputs with
+ * d_k = 128, else the CUDA-core kernel) needs only the 256-byte status word of
+ * that array, for any sizes; sizes beyond what the library indexes (those for which
+ * gdr_prefill_workspace_bytes returns 0) are rejected with GDR_ERR_INVALID_ARG.  The
+ * first call on a device looks up the array's device address with that device
+ * current, so make that first call before any stream capture; a failed lookup is
+ * tried again on the next call.  The call allocates nothing.  After the prefill it
+ * enqueues a one-warp kernel that moves the array's status word into a sticky
+ * per-device word, which gdr_noalloc_status reads; if that launch fails the call
+ * returns GDR_ERR_CUDA although the prefill was already enqueued.  All calls share
+ * the one array: calls that overlap on the GPU (streams without ordering between
+ * them) race. */
 GDR_API gdr_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,
                        const float* alpha, const float* beta, const float* s0,
                        void* o, float* s_final,
                        int B, int T, int H, int dk, int dv,
                        int in_dtype, int out_dtype, int chunk, void* stream);
+
+/* Synchronises `stream`, then reads and clears the sticky status of
+ * gdn_prefill_noalloc on the current device: GDR_ERR_TIMEOUT if a bounded device
+ * wait of any call since the last query gave up (the outputs of those calls are
+ * undefined), GDR_OK otherwise.  No counterpart in the paper; allocates nothing. */
+GDR_API gdr_status gdr_noalloc_status(void* stream);
 
 /* Largest number of tokens per (sequence, head) that gdn_verify / kda_verify take. */
 #define GDR_VERIFY_MAX_TOKENS 16

@@ -9,7 +9,7 @@ import torch
 
 from oracle import gated_delta_rule_backward
 from synth import WORKLOADS, Workload, device_inputs, make_inputs, slice_inputs
-from _util import rel_err, to_np
+from _util import check_elem, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -43,10 +43,17 @@ def _ref(x, do, dsf):
                                      None if dsf is None else dsf.double().numpy())
 
 
-def _check(got, ref, tol, label):
+# per-(batch, head) slicing of each gradient for the element-wise bound: the token
+# tensors [B, T, H, ...] over (0, 2), ds0 [B, H, d_v, d_k] over (0, 1)
+AXES = ((0, 2), (0, 2), (0, 2), (0, 2), (0, 2), (0, 1))
+
+
+def _check(got, ref, tol, label, axes=AXES):
     errs = {n: rel_err(a, b) for n, a, b in zip(NAMES, got, ref)}
     print(label, " ".join(f"{n} {e:.1e}" for n, e in errs.items()))
     assert all(e <= tol for e in errs.values()), errs
+    for n, a, b, ax in zip(NAMES, got, ref, axes):
+        check_elem(a, b, "cc", axes=ax, label=f"{label} {n}")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -135,7 +142,7 @@ def test_full_workload_sampled(name):
         got = [to_np(out[0][0, :, h]), to_np(out[1][0, :, h]), to_np(out[2][0, :, h]),
                to_np(out[3][0, :, h]), to_np(out[4][0, :, h]), to_np(out[5][0, h])]
         ref = [r[0, :, 0] if i < 5 else r[0, 0] for i, r in enumerate(ref)]
-        _check(got, ref, TOL["bf16"], f"{name} head {h}")
+        _check(got, ref, TOL["bf16"], f"{name} head {h}", axes=((),) * 6)
 
 
 def test_rejects_unsupported_and_missing_workspace():

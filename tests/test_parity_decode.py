@@ -6,7 +6,7 @@ import torch
 
 from oracle import decode_step
 from synth import WORKLOADS, Workload, device_inputs, make_inputs, slice_inputs
-from _util import rel_err, to_np
+from _util import check_elem, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -36,9 +36,12 @@ def test_decode_small(mixer, dtype, dk, dv, out):
         torch.cuda.synchronize()
         tol = TOL[dtype] if (out == "f32" or dtype == "f32") else TOL["bf16"]
         assert rel_err(to_np(o), o_ref) <= tol
+        check_elem(to_np(o), o_ref, "cc", axes=(0, 1), bf16_out=o.dtype == torch.bfloat16,
+                   label=f"step {t} o")
     es = rel_err(to_np(state), ref)
     print(f"{mixer} {dtype} {dk}x{dv}: state err {es:.2e}")
     assert es <= TOL[dtype]
+    check_elem(to_np(state), ref, "cc", axes=(0, 1), label="state")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -76,6 +79,8 @@ def test_decode_workload_sampled(mixer):
         es = rel_err(to_np(state[n, h]), ref[i, 0])
         print(f"decode {mixer} {(n, h)}: o {eo:.2e} s {es:.2e}")
         assert eo <= TOL["bf16"] and es <= TOL["bf16"]
+        check_elem(outs[i], o_ref[i], "cc", bf16_out=True, label=f"{(n, h)} o")
+        check_elem(to_np(state[n, h]), ref[i, 0], "cc", label=f"{(n, h)} s")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])

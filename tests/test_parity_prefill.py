@@ -2,7 +2,8 @@
 
 Bar: normwise relative error <= 2e-3 for bf16 inputs and <= 1e-5 for fp32
 inputs, on the outputs and on the final state, for the whole tensor and for
-every (batch, head) slice.
+every (batch, head) slice; and every element within the element-wise bound of
+its precision class (tests/_util.py).
 """
 
 import numpy as np
@@ -11,7 +12,7 @@ import torch
 
 from oracle import gated_delta_rule
 from synth import WORKLOADS, Workload, device_inputs, make_inputs, slice_inputs
-from _util import bf16_round_floor, rel_err, slice_errs, to_np
+from _util import bf16_round_floor, check_elem, rel_err, slice_errs, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -34,13 +35,26 @@ def ref_prefill(x):
     return gated_delta_rule(*args, s0)
 
 
-def check(o, s, o_ref, s_ref, tol, label=""):
+def path_cls(mixer, dtype, dk=128, dv=128):
+    """Precision class of the prefill that serves these parameters: fp32 inputs go to
+    the CUDA-core kernel (1e-5), bf16 inputs to the tensor-core kernels when d_k = 128
+    and to the CUDA-core kernel otherwise."""
+    import gated_delta_rule_79_b200 as g
+    if dtype == "f32":
+        return "f32"
+    tdt = torch.bfloat16
+    return "tc" if g.prefill_path(dk, dv, tdt, mixer == "kda") == "tensor-core" else "cc"
+
+
+def check(o, s, o_ref, s_ref, tol, label="", cls="tc", bf16_out=False):
     eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
     eo_h = slice_errs(o, o_ref, axes=(0, 2))      # per (batch, head) over (T, d_v)
     es_h = slice_errs(s, s_ref, axes=(0, 1))
     print(f"{label} o {eo:.2e} (worst head {eo_h:.2e})  s {es:.2e} (worst head {es_h:.2e})")
     assert eo <= tol and eo_h <= tol, (eo, eo_h)
     assert es <= tol and es_h <= tol, (es, es_h)
+    check_elem(o, o_ref, cls, axes=(0, 2), bf16_out=bf16_out, label=f"{label} o")
+    check_elem(s, s_ref, cls, axes=(0, 1), label=f"{label} s")
 
 
 def test_gdn_sequential_f32_workload():
@@ -49,7 +63,7 @@ def test_gdn_sequential_f32_workload():
     x = make_inputs(w)
     o, s = gpu_prefill("gdn", x)
     o_ref, s_ref = ref_prefill(x)
-    check(o, s, o_ref, s_ref, TOL["f32"], w.name)
+    check(o, s, o_ref, s_ref, TOL["f32"], w.name, cls="f32")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -63,7 +77,8 @@ def test_small_shapes(mixer, dtype, dk, dv, T):
     x = make_inputs(w, seed=T + dk)
     o, s = gpu_prefill(mixer, x, out_dtype=torch.float32)
     o_ref, s_ref = ref_prefill(x)
-    check(o, s, o_ref, s_ref, TOL[dtype], f"{mixer} {dtype} {dk}x{dv} T={T}")
+    check(o, s, o_ref, s_ref, TOL[dtype], f"{mixer} {dtype} {dk}x{dv} T={T}",
+          cls=path_cls(mixer, dtype, dk, dv))
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -76,7 +91,8 @@ def test_stress_gates(mixer, dtype, gates):
     x = make_inputs(w, seed=5, gates=gates)
     o, s = gpu_prefill(mixer, x, out_dtype=torch.float32)
     o_ref, s_ref = ref_prefill(x)
-    check(o, s, o_ref, s_ref, TOL[dtype], f"{mixer} {dtype} gates={gates}")
+    check(o, s, o_ref, s_ref, TOL[dtype], f"{mixer} {dtype} gates={gates}",
+          cls=path_cls(mixer, dtype))
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -116,7 +132,7 @@ def test_full_workload(name, out):
     o_ref, s_ref = ref_prefill(x)
     if out == "bf16":
         print(f"bf16 rounding floor of o: {bf16_round_floor(o_ref):.2e}")
-    check(o, s, o_ref, s_ref, TOL["bf16"], f"{name} out={out}")
+    check(o, s, o_ref, s_ref, TOL["bf16"], f"{name} out={out}", bf16_out=out == "bf16")
 
 
 def test_kda_long_context_sampled():
@@ -146,6 +162,9 @@ def test_kda_long_context_sampled():
         es = rel_err(to_np(s[b, h]), s_ref[i, 0])
         print(f"kda_long slice {(b, h)}: o {eo:.2e} s {es:.2e}")
         assert eo <= TOL["bf16"] and es <= TOL["bf16"]
+        check_elem(to_np(o[b, :, h]), o_ref[i, :, 0], "tc", bf16_out=o.dtype == torch.bfloat16,
+                   label=f"kda_long {(b, h)} o")
+        check_elem(to_np(s[b, h]), s_ref[i, 0], "tc", label=f"kda_long {(b, h)} s")
 
 
 def test_empty_and_state_passthrough():
@@ -196,7 +215,8 @@ def test_in_place_state_carry(mixer):
     o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state)
     torch.cuda.synchronize()
     assert s.data_ptr() == state.data_ptr()
-    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], "alias")
+    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], "alias",
+          bf16_out=o.dtype == torch.bfloat16)
 
 
 @pytest.mark.parametrize("dv", [128, 64])
@@ -242,7 +262,8 @@ def test_both_carries_bf16_out_in_place(carry, mixer, monkeypatch):
     o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state)
     torch.cuda.synchronize()
     assert o.dtype == torch.bfloat16
-    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{carry} carry bf16 in place")
+    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{carry} carry bf16 in place",
+          bf16_out=True)
 
 
 def test_many_chains_take_the_per_head_carry():
@@ -293,5 +314,6 @@ def test_prefill_bf16_out_repeated(mixer):
         g.workspace_status(ws)
         args = [x[k].double().numpy() for k in ("q", "k", "v", "alpha", "beta")]
         o_ref, s_ref = gated_delta_rule(*args, s_ref)
-        check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{mixer} bf16 call {it}")
+        check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{mixer} bf16 call {it}",
+              bf16_out=o.dtype == torch.bfloat16)
         s_ref = to_np(state).astype(np.float64)

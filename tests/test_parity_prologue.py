@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from oracle import apply_prologue, gated_delta_rule, prefill_varlen, verify_steps
-from _util import rel_err, slice_errs, to_np
+from _util import check_elem, rel_err, slice_errs, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -29,6 +29,17 @@ def raw_inputs(mixer, lead, H, dk, dv, dtype, seed, state=True):
     beta = torch.sigmoid(torch.randn(lead + (H,), generator=g))
     x = torch.randn(lead + ((H, dk) if mixer == "kda" else (H,)), generator=g) + 2.0
     return dict(q=q, k=k, v=v, beta=beta, alpha=x)
+
+
+def cls_of(mixer, dtype, dk, dv):
+    """Precision class of the prefill kernel these parameters select (tests/_util.py);
+    with bf16 inputs the CUDA-core paths read q, k that both sides normalised and
+    rounded to bf16 on their own, so they take the "pro" bound."""
+    import gated_delta_rule_79_b200 as g
+    if dtype == "f32":
+        return "f32"
+    return ("tc" if g.prefill_path(dk, dv, torch.bfloat16, mixer == "kda") == "tensor-core"
+            else "pro")
 
 
 def prepared(x, dtype, flags):
@@ -61,6 +72,11 @@ def test_prefill(mixer, dtype, dk, dv, flags):
     eo, es = rel_err(to_np(o), o_ref), rel_err(to_np(s), s_ref)
     print(f"{mixer} {dtype} {dk}x{dv} flags={flags}: o {eo:.2e} s {es:.2e}")
     assert eo <= TOL[dtype] and es <= TOL[dtype]
+    cls = cls_of(mixer, dtype, dk, dv)
+    if cls == "pro" and not flags & 1:
+        cls = "cc"      # q, k given normalised: nothing is rounded on either side
+    check_elem(to_np(o), o_ref, cls, axes=(0, 2), label="o")
+    check_elem(to_np(s), s_ref, cls, axes=(0, 1), label="s")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -78,6 +94,8 @@ def test_prefill_small_workspace_runs_the_cuda_core_kernel(mixer):
     g.workspace_status(ws)
     o_ref, s_ref = gated_delta_rule(*prepared(x, "bf16", BOTH), None)
     assert rel_err(to_np(o), o_ref) <= TOL["bf16"] and rel_err(to_np(s), s_ref) <= TOL["bf16"]
+    check_elem(to_np(o), o_ref, "pro", axes=(0, 2), label="o")
+    check_elem(to_np(s), s_ref, "pro", axes=(0, 1), label="s")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -98,6 +116,9 @@ def test_decode(mixer, dtype, dk, dv):
                                     state.double().numpy())
     assert rel_err(to_np(o), o_ref[:, 0]) <= TOL[dtype]
     assert rel_err(to_np(st), s_ref) <= TOL[dtype]
+    cls = "f32" if dtype == "f32" else "pro"
+    check_elem(to_np(o), o_ref[:, 0], cls, axes=(0, 1), label="o")
+    check_elem(to_np(st), s_ref, cls, axes=(0, 1), label="s")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -114,6 +135,9 @@ def test_verify(mixer):
     o_ref, s_ref = verify_steps(*prepared(x, "bf16", BOTH), state.double().numpy())
     assert slice_errs(to_np(o), o_ref, axes=(0, 2)) <= TOL["bf16"]
     assert max(rel_err(to_np(snaps[i]), s_ref[i]) for i in range(K)) <= TOL["bf16"]
+    check_elem(to_np(o), o_ref, "pro", axes=(0, 2), label="o")
+    for i in range(K):
+        check_elem(to_np(snaps[i]), s_ref[i], "pro", axes=(0, 1), label=f"snapshot {i}")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -134,6 +158,8 @@ def test_varlen(mixer):
     o_ref, p_ref = prefill_varlen(*prepared(x, "bf16", BOTH), cu.numpy(), pool0.double().numpy())
     assert rel_err(to_np(o), o_ref) <= TOL["bf16"]
     assert rel_err(to_np(pool), p_ref) <= TOL["bf16"]
+    check_elem(to_np(o), o_ref, "tc", axes=(1,), label="o")
+    check_elem(to_np(pool), p_ref, "tc", axes=(0, 1), label="pool")
 
 
 def test_unknown_flags_are_rejected():
@@ -175,3 +201,6 @@ def test_full_workload_sampled(name):
         es = rel_err(to_np(s[0, h]), s_ref[0, 0])
         print(f"{name} head {h}: o {eo:.2e} s {es:.2e}")
         assert eo <= TOL["bf16"] and es <= TOL["bf16"]
+        check_elem(to_np(o[0, :, h]), o_ref[0, :, 0], "tc", bf16_out=o.dtype == torch.bfloat16,
+                   label=f"head {h} o")
+        check_elem(to_np(s[0, h]), s_ref[0, 0], "tc", label=f"head {h} s")

@@ -8,7 +8,7 @@ import torch
 
 from oracle import prefill_varlen
 from synth import Workload, make_inputs
-from _util import rel_err, to_np
+from _util import check_elem, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -62,9 +62,11 @@ def test_varlen_ragged(mixer, dv, carry, monkeypatch):
         if b > a:
             eo = rel_err(to_np(o[a:b]), o_ref[a:b])
             assert eo <= TOL, (i, eo)
+            check_elem(to_np(o[a:b]), o_ref[a:b], "tc", axes=(1,), label=f"sequence {i} o")
     for s in range(pool.shape[0]):
         es = rel_err(to_np(pool[s]), p_ref[s])
         assert es <= TOL, (s, es)
+    check_elem(to_np(pool), p_ref, "tc", axes=(0, 1), label="pool")
     print(f"{mixer} dv={dv}: o {rel_err(to_np(o), o_ref):.2e} pool {rel_err(to_np(pool), p_ref):.2e}")
 
 

@@ -7,7 +7,7 @@ import torch
 
 from oracle import verify_steps
 from synth import WORKLOADS, Workload, device_inputs, make_inputs, slice_inputs
-from _util import rel_err, slice_errs, to_np
+from _util import check_elem, rel_err, slice_errs, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +43,9 @@ def test_verify_snapshots(mixer, dtype, dk, dv, K):
     es = max(slice_errs(to_np(snaps[i]), s_ref[i], axes=(0, 1)) for i in range(K))
     print(f"{mixer} {dtype} {dk}x{dv} K={K}: o {eo:.2e} snapshots {es:.2e}")
     assert eo <= TOL[dtype] and es <= TOL[dtype]
+    check_elem(to_np(o), o_ref, "cc", axes=(0, 2), label="o")
+    for i in range(K):
+        check_elem(to_np(snaps[i]), s_ref[i], "cc", axes=(0, 1), label=f"snapshot {i}")
     assert torch.equal(t["s0"], keep)
 
 
@@ -61,6 +64,8 @@ def test_verify_in_place(mixer, K):
     o_ref, s_ref = _ref(x)
     assert rel_err(to_np(o), o_ref) <= TOL["bf16"]
     assert rel_err(to_np(t["s0"]), s_ref[-1]) <= TOL["bf16"]
+    check_elem(to_np(o), o_ref, "cc", axes=(0, 2), bf16_out=True, label="o")
+    check_elem(to_np(t["s0"]), s_ref[-1], "cc", axes=(0, 1), label="state")
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
@@ -86,6 +91,10 @@ def test_verify_workload_sampled(mixer):
         es = rel_err(to_np(snaps[:, n, h]), s_ref[:, 0, 0])
         print(f"{mixer} verify ({n}, {h}): o {eo:.2e} snapshots {es:.2e}")
         assert eo <= TOL["bf16"] and es <= TOL["bf16"]
+        check_elem(to_np(o[n, :, h]), o_ref[0, :, 0], "cc", bf16_out=o.dtype == torch.bfloat16,
+                   label=f"({n}, {h}) o")
+        for i in range(w.T):
+            check_elem(to_np(snaps[i, n, h]), s_ref[i, 0, 0], "cc", label=f"({n}, {h}) snap {i}")
 
 
 def test_verify_rejects_bad_token_counts():
