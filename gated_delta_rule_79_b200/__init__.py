@@ -11,7 +11,7 @@ _PUBLIC = ("gdn_prefill", "kda_prefill", "gdn_decode", "kda_decode", "gdn_verify
            "gdn_prefill_varlen", "kda_prefill_varlen", "gdn_backward", "kda_backward",
            "backward_workspace_bytes", "PROLOGUE_L2NORM_QK", "PROLOGUE_GATE_LOGIT",
            "VERIFY_MAX_TOKENS", "prefill_workspace",
-           "workspace_status", "prefill_path", "timing_start", "timing_stop", "GdrError", "lib", "LIB_PATH", "EXPORTS", "GDR_OK",
+           "workspace_status", "check_status", "noalloc_status", "prefill_path", "timing_start", "timing_stop", "GdrError", "lib", "LIB_PATH", "EXPORTS", "GDR_OK",
            "GDR_ERR_INVALID_ARG", "GDR_ERR_UNSUPPORTED", "GDR_ERR_CUDA", "GDR_ERR_TIMEOUT",
            "GDR_F32", "GDR_BF16", "CHUNK")
 

@@ -14,7 +14,10 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgdr.so")
+# GDR_LIBRARY=checks loads the debug build with device-side index checks
+# (libgdr_checks.so, see build.py) instead of the product library.
+LIB_PATH = os.path.join(_HERE, "libgdr_checks.so" if os.environ.get("GDR_LIBRARY") == "checks"
+                        else "libgdr.so")
 
 GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT = range(5)
 GDR_F32, GDR_BF16 = 0, 1
@@ -22,7 +25,8 @@ CHUNK = 64
 
 EXPORTS = ["gdr_version", "gdr_last_error", "gdr_prefill_workspace_bytes", "gdn_prefill",
            "kda_prefill", "gdn_decode", "kda_decode", "gdr_workspace_status",
-           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_noalloc_status", "gdr_timing_start", "gdr_timing_stop",
+           "gdr_prefill_path", "gdn_prefill_noalloc", "gdr_noalloc_status", "gdr_check_status",
+           "gdr_timing_start", "gdr_timing_stop",
            "gdn_verify", "kda_verify", "gdr_prefill_varlen_workspace_bytes",
            "gdn_prefill_varlen", "kda_prefill_varlen", "gdr_backward_workspace_bytes",
            "gdn_backward", "kda_backward", "gdn_prefill_ex", "kda_prefill_ex", "gdn_decode_ex",
@@ -87,6 +91,8 @@ def _load():
     lib.gdn_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
     lib.gdr_noalloc_status.restype = i
     lib.gdr_noalloc_status.argtypes = [vp]
+    lib.gdr_check_status.restype = i
+    lib.gdr_check_status.argtypes = [vp]
     lib.gdr_prefill_path.restype = i
     lib.gdr_prefill_path.argtypes = [i, i, i, i]
     lib.gdr_workspace_status.restype = i
@@ -434,6 +440,22 @@ def prefill_path(dk, dv, dtype, kda):
     if p < 0:
         raise GdrError(GDR_ERR_UNSUPPORTED, f"no prefill kernel for d_k={dk} d_v={dv}")
     return "tensor-core" if p == 1 else "cuda-core"
+
+
+def check_status(stream=None):
+    """Synchronise and read/clear the device-side index-check word of the checks build
+    (libgdr_checks.so); raises GdrError(GDR_ERR_INVALID_ARG) if a check fired, and
+    GdrError(GDR_ERR_UNSUPPORTED) in the product build, which has no checks."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib.gdr_check_status(_stream(dev, stream)))
+
+
+def noalloc_status(stream=None):
+    """Synchronise and read/clear the sticky status of gdn_prefill_noalloc on the
+    current device; raises GdrError(GDR_ERR_TIMEOUT) if a bounded device wait of a
+    call since the last query gave up."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib.gdr_noalloc_status(_stream(dev, stream)))
 
 
 def workspace_status(workspace, stream=None):

@@ -1,9 +1,12 @@
-"""Build libgdr.so (the C-ABI library) in-tree with nvcc for sm_100a.
+"""Build libgdr.so (the C-ABI library) in-tree with nvcc for sm_100a, and its debug
+twin libgdr_checks.so (the same sources with -DGDR_CHECKS: device-side index checks
+that record a status bit instead of faulting, read with gdr_check_status).
 
-    python -m gated_delta_rule_79_b200.build [--force] [--verbose]
+    python -m gated_delta_rule_79_b200.build [--force] [--verbose] [--checks]
 
-The library is written next to this file so that it travels with the source
-tree; the Python binding loads it from there and fails loudly if it is absent.
+The libraries are written next to this file so that they travel with the source
+tree; the Python binding loads libgdr.so from there (libgdr_checks.so when
+GDR_LIBRARY=checks) and fails loudly if it is absent.
 """
 
 import argparse
@@ -17,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgdr.so")
+LIB_CHECKS = os.path.join(PKG, "libgdr_checks.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -31,20 +35,24 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(LIB):
+def _stale(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) \
         + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force=False, verbose=False, extra_flags=()):
-    """Compile every .cu under csrc/ into libgdr.so (skipped when up to date)."""
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force=False, verbose=False, extra_flags=(), checks=False):
+    """Compile every .cu under csrc/ into libgdr.so, or with checks=True into
+    libgdr_checks.so with -DGDR_CHECKS (skipped when up to date)."""
+    lib = LIB_CHECKS if checks else LIB
+    if not force and not _stale(lib):
+        return lib
+    if checks:
+        extra_flags = ("-DGDR_CHECKS", *extra_flags)
+    objdir = os.path.join(PKG, "_build_checks" if checks else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     procs = []
@@ -65,11 +73,11 @@ def build(force=False, verbose=False, extra_flags=()):
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
@@ -77,6 +85,8 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--checks", action="store_true", help="build libgdr_checks.so instead")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_v else []
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra_flags=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra_flags=extra,
+                checks=a.checks))

@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 
 #include "gdr.h"
@@ -28,6 +29,30 @@ static gdr_status fail(gdr_status s, const char* fmt, ...) {
 }
 
 int report_error(int s, const char* msg) { return fail((gdr_status)s, "%s", msg); }
+
+#ifdef GDR_CHECKS
+static std::mutex g_checks_mu;
+static unsigned int* g_checks[64];
+
+unsigned int* checks_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_checks_mu);
+  if (!g_checks[dev]) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, sizeof(unsigned int)) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, sizeof(unsigned int)) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(p);
+      return nullptr;
+    }
+    g_checks[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_checks[dev];
+}
+#else
+unsigned int* checks_word() { return nullptr; }
+#endif
 
 static gdr_status ok() {
   g_last_error.clear();
@@ -342,6 +367,31 @@ int gdr_prefill_path(int dk, int dv, int in_dtype, int kda) {
   a.in_dtype = in_dtype;
   a.kda = kda != 0;
   return gdr::tc_prefill_supported(a) ? 1 : 0;
+}
+
+gdr_status gdr_check_status(void* stream) {
+#ifdef GDR_CHECKS
+  unsigned int* w = gdr::checks_word();
+  if (!w) return gdr::fail(GDR_ERR_CUDA, "gdr_check_status: no device word for the checks");
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, w, sizeof word, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && word != 0) e = cudaMemsetAsync(w, 0, sizeof word, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return gdr::fail(GDR_ERR_CUDA, "gdr_check_status: %s", cudaGetErrorString(e));
+  if (word != 0)
+    return gdr::fail(GDR_ERR_INVALID_ARG,
+                     "device-side index checks failed (bits 0x%x: 1 chunk location, 2 state "
+                     "index, 4 chunk image, 8 decode/verify row layout); the accesses were "
+                     "skipped", word);
+  return gdr::ok();
+#else
+  (void)stream;
+  return gdr::fail(GDR_ERR_UNSUPPORTED,
+                   "gdr_check_status: this library was built without GDR_CHECKS (the checks "
+                   "build is libgdr_checks.so)");
+#endif
 }
 
 gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream) {

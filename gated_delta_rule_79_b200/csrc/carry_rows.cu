@@ -138,6 +138,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
   const int h = blockIdx.x % H, seq = blockIdx.x / H;
   int first = 0, nchunks = 0;
   chunk_range(m, seq, first, nchunks);
+  if (!dcheck(dv <= 128, m.checks, kCheckImage)) nchunks = 0;
   const int nvb = dv / 32;           // blocks of 32 value columns
 
   if (tid == 0) {
@@ -266,7 +267,8 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
     // =========================== carry warpgroups =====================================
     const int v = tid & 127;         // value row = TMEM lane
     const int hf = tid >> 7;         // which half of the row's columns this thread owns
-    const long srow = (((long)chunk_state_index(m, seq) * H + h) * dv + v) * kDK;
+    const int sidx = chunk_state_index(m, seq);
+    const long srow = (((long)max(sidx, 0) * H + h) * dv + v) * kDK;
     const float4* egl = reinterpret_cast<const float4*>(sm + L_A + WS_EGL);
     uint32_t mphase = 0;
     auto wait_mma = [&]() -> bool {
@@ -327,6 +329,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
     // partial chunk 16 bytes a thread
     auto store_rows = [&](int cc) {
       const ChunkLoc loc = chunk_locate(m, first + cc);
+      if (!loc.valid) return;
       if (!m.cu || loc.L == kC) {
         if (tid == R_STORER) {
           tma_store_4d(&tm_o, smem_u32(stage), 0, h, loc.t0, loc.b);
@@ -358,7 +361,8 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (s0 && v < dv) f = *reinterpret_cast<const float4*>(s0 + srow + 32 * nb + 4 * q);
+          if (s0 && v < dv && sidx >= 0)
+            f = *reinterpret_cast<const float4*>(s0 + srow + 32 * nb + 4 * q);
           x[4 * q] = f.x;
           x[4 * q + 1] = f.y;
           x[4 * q + 2] = f.z;
@@ -478,7 +482,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         float x[32];
         tmem_ld32(tb + tlane + T_S + 32 * nb, x);
         tmem_wait_ld();
-        if (v < dv) {
+        if (v < dv && sidx >= 0) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(s_final + srow + 32 * nb + 4 * q) =

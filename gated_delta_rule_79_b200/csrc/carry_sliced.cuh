@@ -127,6 +127,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
   const int h = sh % H, seq = sh / H;
   int first = 0, nchunks = 0;
   chunk_range(m, seq, first, nchunks);
+  if (!dcheck(h < H && (slice + 1) * NV <= dv, m.checks, kCheckImage)) nchunks = 0;
   const int v0 = slice * NV;
   const uint32_t tlane = (uint32_t)(q4 * 32) << 16;
   const unsigned char* wsb = ws + m.img_base + ((size_t)h * m.nck + first) * kChunkWs;
@@ -230,10 +231,12 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
     if (!ab && nchunks > 0) write_outputs(nchunks - 1);
   } else {
     // =========================== carry warpgroup ======================================
-    const long sbase = ((long)chunk_state_index(m, seq) * H + h) * (long)dv * kDK;
+    const int sidx = chunk_state_index(m, seq);
+    const long sbase = ((long)max(sidx, 0) * H + h) * (long)dv * kDK;
     float st[NV];
 #pragma unroll
-    for (int vv = 0; vv < NV; ++vv) st[vv] = s0 ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
+    for (int vv = 0; vv < NV; ++vv)
+      st[vv] = (s0 && sidx >= 0) ? s0[sbase + (long)(v0 + vv) * kDK + tid] : 0.f;
     auto write_state_operand = [&]() {
 #pragma unroll
       for (int vv = 0; vv < NV; ++vv) st_tile(tSS, NV, vv, tid, st[vv]);
@@ -373,7 +376,7 @@ __device__ __forceinline__ void carry_body(const CUtensorMap* tm_v, const unsign
       fence_before_sync();
       named_bar(1, 128);
     }
-    if (!aborted && s_final) {
+    if (!aborted && s_final && sidx >= 0) {
 #pragma unroll
       for (int vv = 0; vv < NV; ++vv) s_final[sbase + (long)(v0 + vv) * kDK + tid] = st[vv];
     }

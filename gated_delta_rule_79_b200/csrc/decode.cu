@@ -22,6 +22,7 @@
 // The state is streamed (evict-first) because one step's 0.5 GB of state does
 // not fit in L2.
 
+#include "checks.cuh"
 #include "common.cuh"
 #include "launch.h"
 
@@ -41,7 +42,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
               const Tin* __restrict__ v, const float* __restrict__ alpha,
               const float* __restrict__ beta, float* __restrict__ state,
-              Tout* __restrict__ o, int NH, int dv, unsigned pro, int rshift) {
+              Tout* __restrict__ o, int NH, int dv, unsigned pro, int rshift,
+              unsigned int* checks) {
   constexpr int LPR = 8;               // lanes per state row
   constexpr int RPW = 32 / LPR;        // rows per warp instruction
   constexpr int F4 = DK / (4 * LPR);   // float4 pieces per lane per row
@@ -55,6 +57,8 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   const long head = task >> rshift;
   const int part = task & ((1 << rshift) - 1);
   const int rows = dv >> rshift;
+  // the row loop below covers [0, rows) in whole groups of RPW * ITER rows
+  if (!dcheck((rows << rshift) == dv && rows % (RPW * ITER) == 0, checks, kCheckLayout)) return;
   const int sub = lane / LPR;          // which of the 4 rows of an instruction
   const int j = lane % LPR;            // position inside the row group
 
@@ -173,11 +177,11 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
   if (a.out_dtype == GDR_F32)
     decode_kernel<DK, KDA, Tin, float><<<grid, kDecodeWarps * 32, 0, st>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.beta, a.state,
-        (float*)a.o, NH, a.dv, a.pro, rshift);
+        (float*)a.o, NH, a.dv, a.pro, rshift, checks_word());
   else
     decode_kernel<DK, KDA, Tin, __nv_bfloat16><<<grid, kDecodeWarps * 32, 0, st>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.beta, a.state,
-        (__nv_bfloat16*)a.o, NH, a.dv, a.pro, rshift);
+        (__nv_bfloat16*)a.o, NH, a.dv, a.pro, rshift, checks_word());
   return cudaGetLastError();
 }
 

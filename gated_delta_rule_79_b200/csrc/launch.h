@@ -103,6 +103,11 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 // Records `msg` as the calling thread's gdr_last_error() text and returns `s`.
 int report_error(int s, const char* msg);
 
+// GDR_CHECKS build: the current device's word that failed device-side index checks set
+// (checks.cuh), allocated and zeroed on first use; nullptr in the product build (and if
+// that allocation failed).
+unsigned int* checks_word();
+
 // Measurement aid (timing.cu): records an event on `stream` when timing is on.
 // slot -1 marks the start of a prefill call, slot i the end of its i-th kernel.
 void timing_mark(cudaStream_t stream, int slot);

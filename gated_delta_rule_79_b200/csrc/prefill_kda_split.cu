@@ -122,6 +122,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int q4 = warp & 3, hw = warp >> 2;
   const int gc = blockIdx.x % m.nck;
   const int h = blockIdx.x / m.nck;
+  if (!dcheck(h < H, m.checks, kCheckImage)) return;
   const ChunkLoc loc = chunk_locate(m, gc);
   if (!loc.valid) return;            // past the last chunk of the packed sequences
   const int b = loc.b, t0 = loc.t0, L = loc.L;

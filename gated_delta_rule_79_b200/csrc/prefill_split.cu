@@ -47,6 +47,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int tid = threadIdx.x;
   const int gc = blockIdx.x % m.nck;
   const int h = blockIdx.x / m.nck;
+  if (!dcheck(h < H, m.checks, kCheckImage)) return;
   if (!chunk_locate(m, gc).valid) return;   // past the last chunk of the packed sequences
   if (tid == 0) prep_init(ps);
   if (tid < 32) tmem_alloc(&ps.tmem, P_TM_COLS);

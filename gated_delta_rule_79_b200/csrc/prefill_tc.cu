@@ -647,6 +647,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
     m.nchunks = (a.T + GDR_CHUNK - 1) / GDR_CHUNK;
     m.nck = a.B * m.nchunks;
     m.img_base = 256;
+    m.checks = checks_word();
     return a.kda ? launch_prefill_kda_split(a, m, st) : launch_prefill_split(a, m, st);
   }
   if (a.kda) return launch_prefill_kda_tc(a, st);

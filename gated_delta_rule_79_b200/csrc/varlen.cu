@@ -171,6 +171,7 @@ gdr_status prefill_varlen(bool kda, const void* q, const void* k, const void* v,
     m.nchunks = 0;
     m.nck = (int)lay.nck;
     m.img_base = kStatusBytes + lay.idx_bytes;
+    m.checks = checks_word();
     PrefillArgs a{q, k, v, alpha, beta, state, o, state, 1, total, H, dk, dv,
                   in_dtype, out_dtype, kda, workspace, ws_bytes, pro};
     e = kda ? launch_prefill_kda_split(a, m, st) : launch_prefill_split(a, m, st);

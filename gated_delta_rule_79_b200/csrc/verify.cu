@@ -20,6 +20,7 @@
 // and gates, and k_t . q_t, are staged in shared memory per warp.  Bound: HBM, with
 // (1 + K) d_v d_k 4 bytes per (sequence, head) (2 d_v d_k 4 without snapshots).
 
+#include "checks.cuh"
 #include "common.cuh"
 #include "launch.h"
 
@@ -33,7 +34,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
               const float* __restrict__ alpha, const float* __restrict__ beta,
               float* __restrict__ state, float* __restrict__ snaps, Tout* __restrict__ o,
-              int N, int K, int H, int dv, unsigned pro) {
+              int N, int K, int H, int dv, unsigned pro, unsigned int* checks) {
   constexpr int LPR = 8;               // lanes per state row
   constexpr int RPW = 32 / LPR;        // rows per warp instruction
   constexpr int F4 = DK / (4 * LPR);   // float4 pieces per lane per row
@@ -49,6 +50,8 @@ verify_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
   if (task >= 2 * NH) return;
   const long head = task >> 1;                          // n * H + h
   const int rows = dv >> 1;
+  // the row loop below covers [0, rows) in whole groups of RPW * ITER rows
+  if (!dcheck(2 * rows == dv && rows % (RPW * ITER) == 0, checks, kCheckLayout)) return;
   const int rbase = (int)(task & 1) * rows;
   const long n = head / H, h = head % H;
   // per warp: K x (q[DK], k[DK], gate[GA], {beta, k.q, -, -})
@@ -190,14 +193,15 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarps * 32, smem, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                           a.alpha, a.beta, a.state, a.snapshots, (float*)a.o,
-                                          a.N, a.K, a.H, a.dv, a.pro);
+                                          a.N, a.K, a.H, a.dv, a.pro, checks_word());
   } else {
     auto kern = verify_kernel<DK, KDA, Tin, __nv_bfloat16>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarps * 32, smem, st>>>((const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v,
                                           a.alpha, a.beta, a.state, a.snapshots,
-                                          (__nv_bfloat16*)a.o, a.N, a.K, a.H, a.dv, a.pro);
+                                          (__nv_bfloat16*)a.o, a.N, a.K, a.H, a.dv, a.pro,
+                                          checks_word());
   }
   return cudaGetLastError();
 }

@@ -142,6 +142,8 @@ GDR_API gdr_status kda_prefill(const void* q, const void* k, const void* v,
  *   state       [nslots, H, d_v, d_k] fp32 pool: sequence i starts from slot slots[i]
  *               and its final state is written back there (in place); slots is an
  *               int32 DEVICE array [nseq], or NULL for slot i; slots must be distinct
+ *               and within the pool (a negative slot leaves the pool untouched for
+ *               that sequence; the checks build also records it, see gdr_check_status)
  *   o           [total, H, d_v]  out_dtype (written)
  *   workspace   gdr_prefill_varlen_workspace_bytes(...) bytes, 256-byte aligned,
  *               zero-filled at allocation (the status word stays zero between calls)
@@ -362,6 +364,18 @@ GDR_API int gdr_prefill_path(int dk, int dv, int in_dtype, int kda);
  * then undefined), GDR_ERR_INVALID_ARG if a packed-sequence call found its offsets
  * inconsistent (nothing was processed), or GDR_ERR_CUDA. */
 GDR_API gdr_status gdr_workspace_status(void* workspace, size_t ws_bytes, void* stream);
+
+/* Debug aid; the paper has no counterpart.  The library also comes as a debug build,
+ * libgdr_checks.so (compiled with -DGDR_CHECKS), whose kernels test the indices they
+ * derive from device data and from their launch layout before using them: a chunk's
+ * sequence, first token and length against the tensors (bit 1), a batch entry or
+ * state-pool slot (bit 2; slots only for sign, the pool size is not passed), a chunk
+ * image against the workspace (bit 4), a decode / verify thread's rows (bit 8).  A
+ * failed test skips the access and sets its bit in one device word per GPU.  This
+ * call synchronises `stream`, reads and clears that word of the current device and
+ * returns GDR_OK, or GDR_ERR_INVALID_ARG naming the bits.  The product build,
+ * libgdr.so, has no such checks and returns GDR_ERR_UNSUPPORTED without a CUDA call. */
+GDR_API gdr_status gdr_check_status(void* stream);
 
 /* Measurement aid; the paper has no counterpart.  gdr_timing_start() clears the
  * record and makes every later prefill call record a CUDA event on its stream when

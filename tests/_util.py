@@ -18,9 +18,12 @@ class (ELEM_TOL) follow from the arithmetic of the path:
   is a sum of many such roundings, and its largest value over ~1e6 elements sits a
   few standard deviations out, so 8e-3 (16 tf32 units) bounds it with margin.
 * ``cc``: fp32 arithmetic on the CUDA cores (decode, verify, the CUDA-core prefill,
-  the backward) on bf16 or fp32 inputs: normwise ~1e-7, bound 2e-5 per element.
+  the backward) on bf16 or fp32 inputs: normwise ~1e-6.  The chunk-local cumulative
+  log gate G is held in fp32, so a decay e^{G_t - G_j} is off by up to |G| 2^-24
+  relative; the stress gates (alpha = 0, floored at e^-30) drive |G| to several hundred
+  within a chunk, i.e. ~3e-5 per factor.  Bound 1e-4 per element.
 * ``f32``: fp32 inputs through the CUDA-core prefill, held to the 1e-5 normwise bar:
-  the same fp32 arithmetic as ``cc``, bound 2e-5.
+  the same fp32 arithmetic as ``cc``, bound 1e-4.
 * ``pro``: the fused prologue on bf16 inputs through the CUDA-core kernels.  Both
   sides normalise q and k and round them to bf16 on their own, so a rounding decision
   may differ by one bf16 unit (at most 2^-7 of that element of q or k); that element
@@ -40,7 +43,7 @@ import numpy as np
 import torch
 
 NORM_TOL = {"f32": 1e-5, "bf16": 2e-3}
-ELEM_TOL = {"tc": 8e-3, "cc": 2e-5, "f32": 2e-5, "pro": 2e-3}
+ELEM_TOL = {"tc": 8e-3, "cc": 1e-4, "f32": 1e-4, "pro": 2e-3}
 BF16_HALF_UNIT = 2.0 ** -8
 
 

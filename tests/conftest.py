@@ -21,3 +21,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _no_index_check_fired(request):
+    """With the checks build loaded (GDR_LIBRARY=checks), every GPU test must leave the
+    device-side index-check word clear."""
+    yield
+    if os.environ.get("GDR_LIBRARY") != "checks" or "gpu" not in request.keywords:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import gated_delta_rule_79_b200 as g
+    g.check_status()

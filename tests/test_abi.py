@@ -175,3 +175,22 @@ def test_backward_rejects_bad_arguments(g, fn):
     assert call(dO=P + 8) == g.GDR_ERR_INVALID_ARG
     assert call(ws=None) == g.GDR_ERR_INVALID_ARG
     assert call(B=0) == g.GDR_OK
+
+
+def test_checks_build_exports_the_same_symbols(g):
+    """The debug twin (device-side index checks) is built beside the product library and
+    exports every declared symbol too."""
+    path = os.path.join(os.path.dirname(g.LIB_PATH), "libgdr_checks.so")
+    assert os.path.exists(path), "libgdr_checks.so missing: build with --checks"
+    lib = ctypes.CDLL(path)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), f"{name} not exported by libgdr_checks.so"
+
+
+def test_product_build_has_no_device_checks(g):
+    """gdr_check_status answers GDR_ERR_UNSUPPORTED in the product build, without a CUDA
+    call (so this runs on a machine with no GPU)."""
+    if os.environ.get("GDR_LIBRARY") == "checks":
+        pytest.skip("the checks build is loaded")
+    assert g.lib.gdr_check_status(None) == g.GDR_ERR_UNSUPPORTED
+    assert "GDR_CHECKS" in g.lib.gdr_last_error().decode()
