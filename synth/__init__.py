@@ -82,6 +82,10 @@ WORKLOADS = {
     "decode_gdn": Workload("decode_gdn", "gdn", 256, 32, 512, 128, 128, "bf16", "randn", True),
     "decode_kda": Workload("decode_kda", "kda", 256, 32, 512, 128, 128, "bf16", "randn", True),
     "kda_long": Workload("kda_long", "kda", 4, 32, 65536, 128, 128, "bf16", "randn"),
+    # kda_long's batch, heads and entering state over 4096 tokens: the same kernels and
+    # per-chunk traffic (128 chains take the per-head carry) in 1/16 of the memory, for
+    # ncu captures that must stay small
+    "kda_long_t4096": Workload("kda_long_t4096", "kda", 4, 32, 4096, 128, 128, "bf16", "randn"),
     "verify_gdn": Workload("verify_gdn", "gdn", 256, 32, 4, 128, 128, "bf16", "randn",
                            verify=True),
     "verify_kda": Workload("verify_kda", "kda", 256, 32, 4, 128, 128, "bf16", "randn",
