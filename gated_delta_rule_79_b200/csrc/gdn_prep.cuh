@@ -11,7 +11,7 @@
 //
 // The Gram [Q; K] K^T runs as one exact kind::f16 product on the bf16 q, k tiles (the
 // scalar decays e^{G_t - G_j} are applied on read-back); the solve for T runs on the
-// CUDA cores by 16 x 16 blocks.  The image holds [Q (.) e^G; K (.) e^G], e^{G_last}, T,
+// CUDA cores by 16 x 16 blocks (solve64.cuh).  The image holds [Q (.) e^G; K (.) e^G], e^{G_last}, T,
 // (K (.) e^{G_last - G})^T and P as tf32 tiles.
 //
 // prep_chunk is the work of one 128-thread group for one chunk (the kernel is
@@ -24,6 +24,7 @@
 #include "chunk_image.cuh"
 #include "chunkmap.cuh"
 #include "common.cuh"
+#include "solve64.cuh"
 #include "tc.cuh"
 
 namespace gdr {
@@ -35,33 +36,15 @@ constexpr int kC = GDR_CHUNK;
 constexpr int kDK = 128;
 constexpr uint32_t kDrainLimit = 1u << 26;
 
-// [64][64] fp32 scratch with the column index XOR-ed by the row (conflict-free rows
-// and columns), as in the fused kernel.
-__device__ __forceinline__ int sx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
-
-__device__ __forceinline__ void ld4_sx(const float* base, int k, int klo, int c4, float (&e)[4]) {
-  const float4 f = *reinterpret_cast<const float4*>(base + k * 64 + (c4 ^ (k & 28)));
-  const float v[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-  for (int x = 0; x < 4; ++x) e[x] = v[x ^ klo];
-}
-
-// Strictly lower part of A, stored by 16x16 blocks (a, m), m <= a: block index
-// a(a+1)/2 + m, entry (r, i) at r*16 + (i ^ r).
-__device__ __forceinline__ int pa(int a, int m, int r, int i) {
-  return ((a * (a + 1)) / 2 + m) * 256 + r * 16 + (i ^ r);
-}
-
 __device__ __forceinline__ uint64_t kstep(uint64_t desc0, int rows, int ks) {
   return desc0 + (uint64_t)((((ks >> 2) * rows * 128) + ((ks & 3) * 32)) >> 4);
 }
 
 constexpr int P_THREADS = 128;
 constexpr int P_QK = 0;                    // bf16 [128][128] SW128 (q rows 0-63, k 64-127)  32 KB
-// once the Gram has been read, the solve's scratch reuses the q/k tile:
-constexpr int P_X = 0;                     //   X scratch, sx() layout                        16 KB
-constexpr int P_A = 16384;                 //   packed strictly-lower A                       10 KB
-constexpr int P_Z = P_A + 10240;           //   level scratch [3][16][16]                      3 KB
+// once the Gram has been read, the solve's tiles (solve64.cuh layout) reuse the q/k tile:
+constexpr int P_A = 0;                     //   strictly lower A (and the solve's scratch)   16 KB
+constexpr int P_X = 16384;                 //   X = (I + A)^{-1}                               16 KB
 constexpr int P_G = 32768;                 // gate factors: e^{G_t}[64], e^{G_last - G_t}[64], e^{G_last}
 constexpr int P_SMALL = P_G + 1024;
 constexpr int P_SMEM = P_SMALL + 1024 + 1024;   // 36 KB
@@ -101,7 +84,6 @@ __device__ __forceinline__ bool prep_chunk(const CUtensorMap* tm_q, const CUtens
   float* gates = reinterpret_cast<float*>(sm + P_G);
   float* Xs = reinterpret_cast<float*>(sm + P_X);
   float* As = reinterpret_cast<float*>(sm + P_A);
-  float* Zs = reinterpret_cast<float*>(sm + P_Z);
   PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
   uint64_t* tma_bar = reinterpret_cast<uint64_t*>(&ps.tma_bar);
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
@@ -268,107 +250,30 @@ __device__ __forceinline__ bool prep_chunk(const CUtensorMap* tm_q, const CUtens
         *reinterpret_cast<float4*>(ip + swz_off4(t, q, 64)) =
             img::tf32x4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]);
     } else {
+      // row t of A in 16-byte pieces, up to the end of its diagonal block
       const float bt = ps.beta[t];
-      const int a = t >> 4, r = t & 15;
+      const int a = t >> 4;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const int m = j >> 4;
-        if (m <= a) As[pa(a, m, r, j & 15)] = j < t ? bt * d[j] * __expf(gt - ps.g[j]) : 0.f;
+      for (int q = 0; q < 16; ++q) {
+        if ((q >> 2) <= a) {
+          float e[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 4 * q + u;
+            e[u] = j < t ? bt * d[j] * __expf(gt - ps.g[j]) : 0.f;
+          }
+          *reinterpret_cast<float4*>(As + solve64::at4(t, q)) = make_float4(e[0], e[1], e[2], e[3]);
+        }
       }
     }
   }
   fence_before_sync();
   named_bar(BAR, P_THREADS);
-  // ---- X = (I + A)^{-1}: diagonal blocks (one per warp), then three block levels ------------
-  if (lane < 16) {
-    const int a = warp, jl = lane, base = 16 * a;
-    const int bx = base ^ (base & 16);
-    const float* Ab = As + pa(a, a, 0, 0);
-    float x[16];
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) {
-      float a_row[16];
-#pragma unroll
-      for (int i = 0; i < tl; ++i) a_row[i] = Ab[tl * 16 + (i ^ tl)];
-      float acc0 = (tl == jl) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < tl; i += 2) {
-        acc0 = fmaf(-a_row[i], x[i], acc0);
-        if (i + 1 < tl) acc1 = fmaf(-a_row[i + 1], x[i + 1], acc1);
-      }
-      x[tl] = (tl < jl) ? 0.f : acc0 + acc1;
-    }
-    float* Xb = Xs + base * 64 + bx;
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) Xb[tl * 64 + (jl ^ tl)] = x[tl];
-  }
+  // ---- X = (I + A)^{-1}: the diagonal blocks (one per warp), then the column blocks -------
+  solve64::diag(As, Xs, warp, lane);
   named_bar(BAR, P_THREADS);
-#pragma unroll
-  for (int d = 1; d <= 3; ++d) {
-    const int nunits = (4 - d) * 64;           // unit = (block bb, row r, column quad cq)
-    float z[2][4];
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-#pragma unroll
-        for (int m = 0; m < d; ++m)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k = 16 * (bb + m) + i;
-            const float av = As[pa(aa, bb + m, r, i)];
-            float e[4];
-            ld4_sx(Xs, k, i & 3, 16 * bb + 4 * cq, e);
-            z0 = fmaf(av, e[0], z0);
-            z1 = fmaf(av, e[1], z1);
-            z2 = fmaf(av, e[2], z2);
-            z3 = fmaf(av, e[3], z3);
-          }
-        z[n][0] = z0; z[n][1] = z1; z[n][2] = z2; z[n][3] = z3;
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3;
-        *reinterpret_cast<float4*>(&Zs[bb * 256 + r * 16 + 4 * cq]) =
-            make_float4(z[n][0], z[n][1], z[n][2], z[n][3]);
-      }
-    }
-    named_bar(BAR, P_THREADS);
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float xa = Xs[sx(16 * aa + r, 16 * aa + i)];
-          const float4 zz = *reinterpret_cast<const float4*>(&Zs[bb * 256 + i * 16 + 4 * cq]);
-          x0 = fmaf(xa, zz.x, x0);
-          x1 = fmaf(xa, zz.y, x1);
-          x2 = fmaf(xa, zz.z, x2);
-          x3 = fmaf(xa, zz.w, x3);
-        }
-        z[n][0] = -x0; z[n][1] = -x1; z[n][2] = -x2; z[n][3] = -x3;
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int u = tid + P_THREADS * n;
-      if (u < nunits) {
-        const int bb = u >> 6, r = (u >> 2) & 15, cq = u & 3, aa = bb + d;
-        const int row = 16 * aa + r, col = 16 * bb + 4 * cq;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Xs[sx(row, col + e)] = z[n][e];
-      }
-    }
-    named_bar(BAR, P_THREADS);
-  }
+  solve64::offdiag(As, Xs, warp, lane);
+  named_bar(BAR, P_THREADS);
   // ---- T = X Diag(beta) (blocks above the diagonal are zero) -------------------------------
   {
     const int r = tid & 63, half = tid >> 6;
@@ -376,7 +281,7 @@ __device__ __forceinline__ bool prep_chunk(const CUtensorMap* tm_q, const CUtens
 #pragma unroll
     for (int x = 0; x < 32; ++x) {
       const int j = half * 32 + x;
-      xr[x] = ((j >> 4) <= (r >> 4)) ? Xs[sx(r, j)] * ps.beta[j] : 0.f;
+      xr[x] = ((j >> 4) <= (r >> 4)) ? Xs[solve64::at(r, j)] * ps.beta[j] : 0.f;
     }
     unsigned char* it = img + img::WS_T;
 #pragma unroll

@@ -42,6 +42,7 @@
 #include "chunkmap.cuh"
 #include "common.cuh"
 #include "launch.h"
+#include "solve64.cuh"
 #include "tc.cuh"
 #include "tma_host.h"
 
@@ -57,15 +58,6 @@ constexpr float kMaxSpan = 168.f;
 constexpr uint32_t kDrainLimit = 1u << 26;
 constexpr size_t kStatusBytes = 256;
 
-__device__ __forceinline__ int sx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
-
-__device__ __forceinline__ void ld4_sx(const float* base, int k, int klo, int c4, float (&e)[4]) {
-  const float4 f = *reinterpret_cast<const float4*>(base + k * 64 + (c4 ^ (k & 28)));
-  const float v[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-  for (int x = 0; x < 4; ++x) e[x] = v[x ^ klo];
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
 
@@ -75,8 +67,8 @@ __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p 
 
 constexpr int P_THREADS = 256;
 constexpr int P_L = 0;            // L = [Q; K] (.) e^{G - Gm}, tf32 [128][128] SW128      64 KB
-                                  //   after the Gram: A (sx) | X (sx) | level scratch
-constexpr int P_AS = 0, P_XS = 16384, P_ZS = 32768;
+                                  //   after the Gram: A | X (solve64.cuh layout)
+constexpr int P_AS = 0, P_XS = 16384;
 constexpr int P_R = 65536;        // R = K (.) e^{Gm - G}, tf32 [64][128] SW128            32 KB
                                   //   after the Gram: G [64 t][128 c] for wide channels
 constexpr int P_SMALL = P_R + 32768;
@@ -112,7 +104,6 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   unsigned char* tR = sm + P_R;
   float* As = reinterpret_cast<float*>(sm + P_AS);
   float* Xs = reinterpret_cast<float*>(sm + P_XS);
-  float* Zs = reinterpret_cast<float*>(sm + P_ZS);
   float* Gw = reinterpret_cast<float*>(tR);
   PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(&ps.mma_bar);
@@ -374,82 +365,25 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
         *reinterpret_cast<float4*>(ip + swz_off4(t, 8 * hw + x, 64)) = tf32x4(e[0], e[1], e[2], e[3]);
       }
     } else {
+      // row t of A, columns 32 hw .. 32 hw + 31, in 16-byte pieces
 #pragma unroll
-      for (int x = 0; x < 32; ++x) As[sx(t, 32 * hw + x)] = (32 * hw + x) < t ? bt * d[x] : 0.f;
+      for (int x = 0; x < 8; ++x) {
+        float e[4];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) e[y] = (32 * hw + 4 * x + y) < t ? bt * d[4 * x + y] : 0.f;
+        *reinterpret_cast<float4*>(As + solve64::at4(t, 8 * hw + x)) =
+            make_float4(e[0], e[1], e[2], e[3]);
+      }
     }
   }
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, P_TM_COLS);
-  // ---- 6. X = (I + A)^{-1}: diagonal 16x16 blocks (one per warp), then three block levels ---
-  if (warp < 4 && lane < 16) {
-    const int base = 16 * warp, jl = lane;
-    const int bx = base ^ (base & 16);
-    const float* Ab = As + base * 64 + bx;
-    float x[16];
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) {
-      float a_row[16];
-#pragma unroll
-      for (int i = 0; i < tl; ++i) a_row[i] = Ab[tl * 64 + (i ^ tl)];
-      float acc0 = (tl == jl) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < tl; i += 2) {
-        acc0 = fmaf(-a_row[i], x[i], acc0);
-        if (i + 1 < tl) acc1 = fmaf(-a_row[i + 1], x[i + 1], acc1);
-      }
-      x[tl] = (tl < jl) ? 0.f : acc0 + acc1;
-    }
-    float* Xb = Xs + base * 64 + bx;
-#pragma unroll
-    for (int tl = 0; tl < 16; ++tl) Xb[tl * 64 + (jl ^ tl)] = x[tl];
-  }
+  // ---- 6. X = (I + A)^{-1}: the diagonal blocks (warps 0-3), then the column blocks -------
+  if (warp < 4) solve64::diag(As, Xs, warp, lane);
   __syncthreads();
-  {
-    const int bb = tid >> 6, r = (tid >> 2) & 15, cq = tid & 3;
-#pragma unroll
-    for (int d = 1; d <= 3; ++d) {
-      const bool act = bb < 4 - d;
-      const int aa = bb + d;
-      if (act) {
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
-#pragma unroll
-        for (int m = 0; m < d; ++m) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int kk = 16 * (bb + m) + i;
-            const float a = As[sx(16 * aa + r, kk)];
-            float e[4];
-            ld4_sx(Xs, kk, i & 3, 16 * bb + 4 * cq, e);
-            z0 = fmaf(a, e[0], z0);
-            z1 = fmaf(a, e[1], z1);
-            z2 = fmaf(a, e[2], z2);
-            z3 = fmaf(a, e[3], z3);
-          }
-        }
-        *reinterpret_cast<float4*>(&Zs[bb * 256 + r * 16 + 4 * cq]) = make_float4(z0, z1, z2, z3);
-      }
-      __syncthreads();
-      if (act) {
-        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float xa = Xs[sx(16 * aa + r, 16 * aa + i)];
-          const float4 zz = *reinterpret_cast<const float4*>(&Zs[bb * 256 + i * 16 + 4 * cq]);
-          x0 = fmaf(xa, zz.x, x0);
-          x1 = fmaf(xa, zz.y, x1);
-          x2 = fmaf(xa, zz.z, x2);
-          x3 = fmaf(xa, zz.w, x3);
-        }
-        const int row = 16 * aa + r, col = 16 * bb + 4 * cq;
-        Xs[sx(row, col + 0)] = -x0;
-        Xs[sx(row, col + 1)] = -x1;
-        Xs[sx(row, col + 2)] = -x2;
-        Xs[sx(row, col + 3)] = -x3;
-      }
-      __syncthreads();
-    }
-  }
+  if (warp < 4) solve64::offdiag(As, Xs, warp, lane);
+  __syncthreads();
   // ---- 7. T = X Diag(beta) to the image (blocks above the diagonal are zero) ------------------
   {
     const int r = tid & 63, qq = tid >> 6;
@@ -460,7 +394,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
         const int j = 16 * qq + 4 * x + y;
-        e[y] = (qq <= (r >> 4)) ? Xs[sx(r, j)] * ps.beta[j] : 0.f;
+        e[y] = (qq <= (r >> 4)) ? Xs[solve64::at(r, j)] * ps.beta[j] : 0.f;
       }
       *reinterpret_cast<float4*>(it + swz_off4(r, 4 * qq + x, 64)) = tf32x4(e[0], e[1], e[2], e[3]);
     }
