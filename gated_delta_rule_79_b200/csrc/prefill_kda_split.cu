@@ -428,7 +428,6 @@ cudaError_t launch_kda_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStre
   timing_mark(stream, 0);
   e = launch_chunk_carry(a, m, lim, stream);
   e = cudaGetLastError();
-  if (e == cudaSuccess) timing_mark(stream, 1);
   return e;
 }
 
