@@ -528,23 +528,7 @@ def time_e2e(w, dev, steps, warmup, seed):
                snapshots=snaps, o=o)
             o_host.copy_(o, non_blocking=True)
     else:
-        fn = g.kda_prefill if w.mixer == "kda" else g.gdn_prefill
-        dbuf = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
-        ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev)
-        o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
-        s = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
-        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        s_host = torch.empty(s.shape, dtype=s.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in dbuf.values())
-        d2h = o.numel() * 2 + s.numel() * 4
-
-        def step():
-            for key in dbuf:
-                dbuf[key].copy_(host[key], non_blocking=True)
-            fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], dbuf.get("s0"),
-               o=o, s_final=s, workspace=ws, prologue=w.prologue)
-            o_host.copy_(o, non_blocking=True)
-            s_host.copy_(s, non_blocking=True)
+        return _e2e_prefill_overlapped(w, dev, steps, warmup, x, host)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -557,6 +541,74 @@ def time_e2e(w, dev, steps, warmup, seed):
     ms = a.elapsed_time(b) / steps
     return {"value": tokens(w) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
+
+
+def _e2e_prefill_overlapped(w, dev, steps, warmup, x, host):
+    """Prefill through the public API with pinned host buffers, the copies overlapped with
+    the computation: two device buffer sets; step i's inputs go host->device on one copy
+    stream while step i-1 computes, and step i-2's outputs go device->host on another.
+    Every step copies all of its inputs in and all of its outputs (o and the final state)
+    out inside the timed region, which runs from an event before the first copy to one
+    after the last copy out."""
+    import gated_delta_rule_79_b200 as g
+    fn = g.kda_prefill if w.mixer == "kda" else g.gdn_prefill
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    keys = [k for k, v in x.items() if v is not None]
+    sets = [{k: torch.empty_like(x[k]) for k in keys} for _ in range(2)]
+    outs = [(torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev),
+             torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev))
+            for _ in range(2)]
+    o_host = torch.empty(outs[0][0].shape, dtype=torch.bfloat16).pin_memory()
+    s_host = torch.empty(outs[0][1].shape, dtype=torch.float32).pin_memory()
+    ws, _ = g.prefill_workspace(w.B, w.T, w.H, w.dk, w.dv, w.mixer == "kda", dev, stream=comp)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    h2d = sum(sets[0][k].numel() * sets[0][k].element_size() for k in keys)
+    d2h = outs[0][0].numel() * 2 + outs[0][1].numel() * 4
+
+    def step(i):
+        b = i % 2
+        if i >= 2:
+            up.wait_event(ev_done[b])          # step i-2 has read this input set
+        with torch.cuda.stream(up):
+            for k in keys:
+                sets[b][k].copy_(host[k], non_blocking=True)
+            ev_in[b].record(up)
+        comp.wait_event(ev_in[b])
+        if i >= 2:
+            comp.wait_event(ev_out[b])         # step i-2's outputs have been copied out
+        d = sets[b]
+        fn(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d.get("s0"), o=outs[b][0],
+           s_final=outs[b][1], workspace=ws, prologue=w.prologue)
+        ev_done[b].record(comp)
+        down.wait_event(ev_done[b])
+        with torch.cuda.stream(down):
+            o_host.copy_(outs[b][0], non_blocking=True)
+            s_host.copy_(outs[b][1], non_blocking=True)
+            ev_out[b].record(down)
+
+    def run(first, n):
+        for i in range(first, first + n):
+            step(i)
+        for b in range(2):
+            comp.wait_event(ev_out[b])
+
+    run(0, warmup)
+    torch.cuda.synchronize(dev)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    up.wait_event(a)
+    down.wait_event(a)
+    run(warmup, steps)
+    e.record(comp)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(e) / steps
+    return {"value": tokens(w) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+            "copies": "overlapped: host->device of step i, compute of step i-1 and "
+                      "device->host of step i-2 on three streams"}
 
 
 # ----------------------------------------------------------------------------------------

@@ -19,10 +19,11 @@ namespace gdr {
 //
 // A dense batch of few long chains may instead take the two-segment carry (each chain's
 // chunks in two halves run at once by three per-head CTAs, then carry_segfix.cu adds the
-// first half's state to the second half): when its three CTAs per chain fit one wave,
-// each chain has at least kSegMinChunks chunks and the workspace holds its buffers
-// (gdr_prefill_workspace_bytes counts them).  GDR_CARRY=seg picks it whenever the
-// workspace allows.
+// first half's state to the second half) when the workspace holds its buffers
+// (gdr_prefill_workspace_bytes counts them).  It is not picked on its own: on the B1 H32
+// T4096 prefills it measured 0.143 ms (the per-head carry over 32 chunks) + 0.040 ms (the
+// fix-up) against 0.173 ms for the value-sliced carry.  GDR_CARRY=seg picks it.
+constexpr bool kSegAuto = false;
 constexpr int kSegMinChunks = 16;
 
 cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
@@ -46,7 +47,7 @@ cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t
     rows = false;
   } else {
     rows = chains * (a.dv / 32) > sms;
-    seg = !rows && seg_ok && 3 * chains <= sms && m.nchunks >= kSegMinChunks;
+    seg = kSegAuto && !rows && seg_ok && 3 * chains <= sms && m.nchunks >= kSegMinChunks;
   }
   if (seg) {
     SegmentBuffers sb;

@@ -355,22 +355,3 @@ def test_two_segment_carry_bf16_out_in_place(mixer, monkeypatch):
     assert o.dtype == torch.bfloat16
     check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], "two-segment bf16 in place",
           bf16_out=True)
-
-
-def test_two_segment_carry_is_the_few_chains_choice():
-    """With the full workspace, B x H x 3 CTAs within one wave and at least 16 chunks a
-    chain, the call takes the two-segment carry: its result equals the forced one bit
-    for bit, and differs (by rounding) from the value-sliced carry's."""
-    import os
-    w = Workload("segpick", "gdn", 1, 8, 1500, 128, 128, "bf16", "randn")
-    x = make_inputs(w, seed=99, gates="slow")
-    auto = gpu_prefill("gdn", x, out_dtype=torch.float32)
-    os.environ["GDR_CARRY"] = "seg"
-    try:
-        forced = gpu_prefill("gdn", x, out_dtype=torch.float32)
-        os.environ["GDR_CARRY"] = "sliced"
-        sliced = gpu_prefill("gdn", x, out_dtype=torch.float32)
-    finally:
-        del os.environ["GDR_CARRY"]
-    assert np.array_equal(auto[0], forced[0]) and np.array_equal(auto[1], forced[1])
-    assert not np.array_equal(auto[0], sliced[0])
