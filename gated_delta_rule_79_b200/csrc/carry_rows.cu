@@ -131,14 +131,18 @@ __device__ __forceinline__ void mma_tf32_ta_1(uint32_t tmem_d, uint32_t tmem_a, 
 // outputs to tm_w slab chain and final state to seg_state[1]; kind 2: the second half
 // with identity state rows and zero values, outputs to tm_w slab BH + chain and final
 // state, transposed, to seg_state[2]).  seg_state holds 3 x BH states of 128 x 128 fp32.
-template <typename Tout>
-__global__ void __launch_bounds__(R_THREADS, 1)
-row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                 const __grid_constant__ CUtensorMap tm_w,
-                 const unsigned char* __restrict__ ws, const float* __restrict__ s0,
-                 Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m, int H,
-                 int dv, unsigned int* __restrict__ status, uint32_t spin_limit, int nseg,
-                 float* __restrict__ seg_state) {
+// The body of one carry CTA of kind KIND (0 when SEG is false), specialised so that the
+// one-segment carry compiles with none of the two-segment paths and each two-segment CTA
+// runs only its own.
+template <typename Tout, int KIND, bool SEG>
+__device__ __forceinline__ void row_carry_body(
+    const CUtensorMap& tm_v, const CUtensorMap& tm_o, const CUtensorMap& tm_w,
+    const unsigned char* __restrict__ ws, const float* __restrict__ s0, Tout* __restrict__ o,
+    float* __restrict__ s_final, const ChunkMap& m, int H, int dv,
+    unsigned int* __restrict__ status, uint32_t spin_limit, float* __restrict__ seg_state,
+    int chain) {
+  constexpr int nseg = SEG ? 2 : 1;
+  constexpr int kind = KIND;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + padb;
@@ -153,8 +157,6 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
   uint64_t* ld_done = reinterpret_cast<uint64_t*>(&cs.ld_done);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kind = nseg == 2 ? (int)(blockIdx.x % 3) : 0;
-  const int chain = nseg == 2 ? (int)(blockIdx.x / 3) : (int)blockIdx.x;
   const int h = chain % H, seq = chain / H;
   int first = 0, nchunks = 0;
   chunk_range(m, seq, first, nchunks);
@@ -169,8 +171,8 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
       nchunks -= n0;
     }
   }
-  const bool ident = kind == 2;      // identity state rows, zero values
-  const bool to_ws = kind != 0;      // fp32 outputs to the workspace slab
+  constexpr bool ident = kind == 2;  // identity state rows, zero values
+  constexpr bool to_ws = kind != 0;  // fp32 outputs to the workspace slab
   const int nvb = ident ? 0 : dv / 32;   // blocks of 32 value columns loaded per chunk
 
   if (tid == 0) {
@@ -350,7 +352,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
             const int t = 32 * half + x;
-            if (to_ws)   // the identity rows' outputs are a tf32 operand of the fix-up
+            if constexpr (to_ws)   // the identity rows' outputs: a tf32 operand of the fix-up
               *reinterpret_cast<float*>(stage + t * rowb + 4 * v) = ident ? to_tf32(ov[x]) : ov[x];
             else if constexpr (sizeof(Tout) == 2)
               *reinterpret_cast<__nv_bfloat16*>(stage + t * rowb + 2 * v) = __float2bfloat16_rn(ov[x]);
@@ -367,7 +369,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
     auto store_rows = [&](int cc) {
       const ChunkLoc loc = chunk_locate(m, first + cc);
       if (!loc.valid) return;
-      if (to_ws) {
+      if constexpr (to_ws) {
         // the segment's chunk cc, whole, to its slab of the workspace ([64 cc + t][128])
         if (tid == R_STORER) {
           tma_store_4d(&tm_w, smem_u32(stage), 0, 0, kC * cc, (kind - 1) * BHn + chain);
@@ -412,7 +414,7 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
           x[4 * q + 1] = f.y;
           x[4 * q + 2] = f.z;
           x[4 * q + 3] = f.w;
-          if (ident) {
+          if constexpr (ident) {
             // row v of the identity
 #pragma unroll
             for (int e = 0; e < 4; ++e) x[4 * q + e] = (32 * nb + 4 * q + e == v) ? 1.f : 0.f;
@@ -537,8 +539,8 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
         float x[32];
         tmem_ld32(tb + tlane + T_S + 32 * nb, x);
         tmem_wait_ld();
-        if (nseg == 2 && kind != 1) round32(x);   // tf32 operands of the fix-up's products
-        if (ident) {
+        if constexpr (SEG && kind != 1) round32(x);   // tf32 operands of the fix-up's products
+        if constexpr (ident) {
 #pragma unroll
           for (int q = 0; q < 32; ++q) dst[(size_t)(32 * nb + q) * kDK + v] = x[q];
         } else if (v < dv && sidx >= 0) {
@@ -555,6 +557,33 @@ row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, T_COLS);
+}
+
+// nseg = 1: one CTA per (sequence, head) chain.  nseg = 2: three CTAs per chain, kind =
+// blockIdx.x % 3 (see row_carry_body).
+template <typename Tout, bool SEG>
+__global__ void __launch_bounds__(R_THREADS, 1)
+row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const __grid_constant__ CUtensorMap tm_w,
+                 const unsigned char* __restrict__ ws, const float* __restrict__ s0,
+                 Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m, int H,
+                 int dv, unsigned int* __restrict__ status, uint32_t spin_limit,
+                 float* __restrict__ seg_state) {
+  if constexpr (!SEG) {
+    row_carry_body<Tout, 0, false>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
+                                   spin_limit, seg_state, (int)blockIdx.x);
+  } else {
+    const int kind = (int)(blockIdx.x % 3), chain = (int)(blockIdx.x / 3);
+    if (kind == 0)
+      row_carry_body<Tout, 0, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
+                                    spin_limit, seg_state, chain);
+    else if (kind == 1)
+      row_carry_body<Tout, 1, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
+                                    spin_limit, seg_state, chain);
+    else
+      row_carry_body<Tout, 2, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
+                                    spin_limit, seg_state, chain);
+  }
 }
 
 }  // namespace
@@ -578,12 +607,12 @@ cudaError_t launch_rows_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim,
   } else {
     mw = mo;   // not read
   }
-  auto carry = row_carry_kernel<Tout>;
+  auto carry = seg ? row_carry_kernel<Tout, true> : row_carry_kernel<Tout, false>;
   cudaError_t e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, L_SMEM);
   if (e != cudaSuccess) return e;
   carry<<<BH * (seg ? 3 : 1), R_THREADS, L_SMEM, stream>>>(
       mv, mo, mw, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H, a.dv,
-      (unsigned int*)a.workspace, lim, seg ? 2 : 1, seg ? seg->states : nullptr);
+      (unsigned int*)a.workspace, lim, seg ? seg->states : nullptr);
   return cudaGetLastError();
 }
 
