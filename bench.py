@@ -269,14 +269,6 @@ class PrefillRunner:
         self.launches_per_step = len(self.kernels)
         self.l2_note = f"{len(self.sets)} rotating input sets of {set_bytes / 2**20:.0f} MiB (> 3x L2)"
 
-    def timed_kernels(self, nslots):
-        """The kernels of one call as the library's timing marks saw them: three with the
-        two-segment carry (prep, two-segment row_carry_kernel, segment_fixup_kernel)."""
-        if self.path == "tensor-core" and nslots == 3:
-            self.kernels = [f"{self.w.mixer}_chunk_prep_kernel",
-                            "row_carry_kernel (two segments)", "segment_fixup_kernel"]
-            self.launches_per_step = 3
-
     def step(self, i):
         x = self.sets[i % len(self.sets)]
         self.fn(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["s0"],
@@ -779,8 +771,6 @@ def run_ours(w, steps, warmup, dev, rank, world, active, peaks, peak_kind, e2e=T
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
                 "launch_ms": launch_ms}
     if kernel_ms:
-        if hasattr(runner, "timed_kernels"):
-            runner.timed_kernels(len(kernel_ms))
         # one "launch" of the roofline is one call of the path; its kernels, timed
         # with events on the launching stream over the same timed steps:
         tot = sum(kernel_ms)

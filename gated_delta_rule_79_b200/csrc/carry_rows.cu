@@ -38,17 +38,6 @@
 // The value-sliced carry (carry_sliced.cu) spreads one head over several SMs instead; it
 // wins when there are too few (sequence, head) chains to fill the GPU.
 //
-// Two segments (nseg = 2, few long chains): the state after a run of chunks is affine in
-// the state before it, S_out = S_in M + B (M the product of the chunks' transitions, B what
-// the run makes from a zero state), and each output is affine in it as well.  So each
-// chain's chunks are cut into two halves run at once by three CTAs: the first half from
-// the given state (outputs final, its final state is the second half's entering state
-// S_in), the second half from a zero state (outputs and final state B to the
-// workspace in fp32), and the second half again with the identity as its state rows and
-// zero values, which yields M (its final state, stored transposed) and, as its outputs,
-// the rows M_t q_t through which S_in reaches output t.  carry_segfix.cu then adds
-// S_in M_t q_t to the second half's outputs and forms S_in M + B.
-//
 // Precision: kind::tf32 products with every operand rounded to nearest.  Waits are
 // bounded; a give-up records GDR_ERR_TIMEOUT in the workspace status word, drains what
 // was issued, frees tensor memory and ends the CTA.
@@ -126,23 +115,12 @@ __device__ __forceinline__ void mma_tf32_ta_1(uint32_t tmem_d, uint32_t tmem_a, 
       : "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1 : 0));
 }
 
-// nseg = 1: one CTA per (sequence, head) chain.  nseg = 2: three CTAs per chain (kind 0:
-// the first half from s0, final state to seg_state[0]; kind 1: the second half from zero,
-// outputs to tm_w slab chain and final state to seg_state[1]; kind 2: the second half
-// with identity state rows and zero values, outputs to tm_w slab BH + chain and final
-// state, transposed, to seg_state[2]).  seg_state holds 3 x BH states of 128 x 128 fp32.
-// The body of one carry CTA of kind KIND (0 when SEG is false), specialised so that the
-// one-segment carry compiles with none of the two-segment paths and each two-segment CTA
-// runs only its own.
-template <typename Tout, int KIND, bool SEG>
-__device__ __forceinline__ void row_carry_body(
-    const CUtensorMap& tm_v, const CUtensorMap& tm_o, const CUtensorMap& tm_w,
-    const unsigned char* __restrict__ ws, const float* __restrict__ s0, Tout* __restrict__ o,
-    float* __restrict__ s_final, const ChunkMap& m, int H, int dv,
-    unsigned int* __restrict__ status, uint32_t spin_limit, float* __restrict__ seg_state,
-    int chain) {
-  constexpr int nseg = SEG ? 2 : 1;
-  constexpr int kind = KIND;
+template <typename Tout>
+__global__ void __launch_bounds__(R_THREADS, 1)
+row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const unsigned char* __restrict__ ws, const float* __restrict__ s0,
+                 Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m, int H,
+                 int dv, unsigned int* __restrict__ status, uint32_t spin_limit) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t padb = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + padb;
@@ -157,23 +135,11 @@ __device__ __forceinline__ void row_carry_body(
   uint64_t* ld_done = reinterpret_cast<uint64_t*>(&cs.ld_done);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = chain % H, seq = chain / H;
+  const int h = blockIdx.x % H, seq = blockIdx.x / H;
   int first = 0, nchunks = 0;
   chunk_range(m, seq, first, nchunks);
   if (!dcheck(dv <= 128, m.checks, kCheckImage)) nchunks = 0;
-  if (nseg == 2) {
-    // the first ceil(n/2) chunks are the first segment
-    const int n0 = (nchunks + 1) >> 1;
-    if (kind == 0) {
-      nchunks = n0;
-    } else {
-      first += n0;
-      nchunks -= n0;
-    }
-  }
-  constexpr bool ident = kind == 2;  // identity state rows, zero values
-  constexpr bool to_ws = kind != 0;  // fp32 outputs to the workspace slab
-  const int nvb = ident ? 0 : dv / 32;   // blocks of 32 value columns loaded per chunk
+  const int nvb = dv / 32;           // blocks of 32 value columns
 
   if (tid == 0) {
     for (int g = 0; g < NG; ++g) {
@@ -303,9 +269,6 @@ __device__ __forceinline__ void row_carry_body(
     const int hf = tid >> 7;         // which half of the row's columns this thread owns
     const int sidx = chunk_state_index(m, seq);
     const long srow = (((long)max(sidx, 0) * H + h) * dv + v) * kDK;
-    const int BHn = m.nseq * H;
-    // rows a segment CTA keeps: value rows (kinds 0, 1) or all 128 identity rows (kind 2)
-    const int nrows = ident ? kDK : dv;
     const float4* egl = reinterpret_cast<const float4*>(sm + L_A + WS_EGL);
     uint32_t mphase = 0;
     auto wait_mma = [&]() -> bool {
@@ -331,7 +294,7 @@ __device__ __forceinline__ void row_carry_body(
       tmem_st32(tb + tlane + T_SR + 32 * nb, x);
     };
     const unsigned char* vrow = sm + L_V + (v >> 5) * 4096 + (v & 31) * 2;
-    const int rowb = to_ws ? kDK * 4 : dv * (int)sizeof(Tout);
+    const int rowb = dv * (int)sizeof(Tout);
     unsigned char* stage = sm + L_O;
     // O^T of chunk cc (D buffer cc & 1, columns 0-63) into the staging tile, one value
     // column per thread (the tile's previous store has read it: see the end of a chunk).
@@ -348,13 +311,11 @@ __device__ __forceinline__ void row_carry_body(
         float ov[32];
         tmem_ld32(tb + tlane + T_D + 128 * po + 32 * half, ov);
         tmem_wait_ld();
-        if (v < nrows) {
+        if (v < dv) {
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
             const int t = 32 * half + x;
-            if constexpr (to_ws)   // the identity rows' outputs: a tf32 operand of the fix-up
-              *reinterpret_cast<float*>(stage + t * rowb + 4 * v) = ident ? to_tf32(ov[x]) : ov[x];
-            else if constexpr (sizeof(Tout) == 2)
+            if constexpr (sizeof(Tout) == 2)
               *reinterpret_cast<__nv_bfloat16*>(stage + t * rowb + 2 * v) = __float2bfloat16_rn(ov[x]);
             else
               *reinterpret_cast<float*>(stage + t * rowb + 4 * v) = ov[x];
@@ -369,14 +330,6 @@ __device__ __forceinline__ void row_carry_body(
     auto store_rows = [&](int cc) {
       const ChunkLoc loc = chunk_locate(m, first + cc);
       if (!loc.valid) return;
-      if constexpr (to_ws) {
-        // the segment's chunk cc, whole, to its slab of the workspace ([64 cc + t][128])
-        if (tid == R_STORER) {
-          tma_store_4d(&tm_w, smem_u32(stage), 0, 0, kC * cc, (kind - 1) * BHn + chain);
-          bulk_commit();
-        }
-        return;
-      }
       if (!m.cu || loc.L == kC) {
         if (tid == R_STORER) {
           tma_store_4d(&tm_o, smem_u32(stage), 0, h, loc.t0, loc.b);
@@ -408,17 +361,12 @@ __device__ __forceinline__ void row_carry_body(
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (kind == 0 && s0 && v < dv && sidx >= 0)
+          if (s0 && v < dv && sidx >= 0)
             f = *reinterpret_cast<const float4*>(s0 + srow + 32 * nb + 4 * q);
           x[4 * q] = f.x;
           x[4 * q + 1] = f.y;
           x[4 * q + 2] = f.z;
           x[4 * q + 3] = f.w;
-          if constexpr (ident) {
-            // row v of the identity
-#pragma unroll
-            for (int e = 0; e < 4; ++e) x[4 * q + e] = (32 * nb + 4 * q + e == v) ? 1.f : 0.f;
-          }
         }
         store_state(nb, x, nchunks > 0);
       }
@@ -454,10 +402,9 @@ __device__ __forceinline__ void row_carry_body(
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const float vv = (!ident && v < dv)
-                               ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                     vrow + (32 * hf + x) * 64))
-                               : 0.f;
+          const float vv = v < dv ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                        vrow + (32 * hf + x) * 64))
+                                  : 0.f;
           y[x] = to_tf32(vv - y[x]);
         }
         tmem_st32(tb + tlane + tD + 64 + 32 * hf, y);
@@ -527,26 +474,18 @@ __device__ __forceinline__ void row_carry_body(
       named_bar(1, R_CARRY);
       store_rows(nchunks - 1);
     }
-    if (!aborted && (s_final || nseg == 2)) {
-      // the last pass left the state undecayed in S.  Segments: kinds 0 and 1 store their
-      // rows to seg_state[kind]; kind 2 stores row v of M as column v of seg_state[2].
-      float* dst = nseg == 2 ? seg_state + ((size_t)kind * BHn + chain) * kDK * kDK
-                             : s_final + srow;
-      if (nseg == 2 && !ident) dst += (size_t)v * kDK;
+    if (!aborted && s_final) {
+      // the last pass left the state undecayed in S
 #pragma unroll
       for (int nh = 0; nh < 2; ++nh) {
         const int nb = 2 * hf + nh;
         float x[32];
         tmem_ld32(tb + tlane + T_S + 32 * nb, x);
         tmem_wait_ld();
-        if constexpr (SEG && kind != 1) round32(x);   // tf32 operands of the fix-up's products
-        if constexpr (ident) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) dst[(size_t)(32 * nb + q) * kDK + v] = x[q];
-        } else if (v < dv && sidx >= 0) {
+        if (v < dv && sidx >= 0) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(dst + 32 * nb + 4 * q) =
+            *reinterpret_cast<float4*>(s_final + srow + 32 * nb + 4 * q) =
                 make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         }
       }
@@ -559,67 +498,32 @@ __device__ __forceinline__ void row_carry_body(
   if (warp == 0) tmem_dealloc(tb, T_COLS);
 }
 
-// nseg = 1: one CTA per (sequence, head) chain.  nseg = 2: three CTAs per chain, kind =
-// blockIdx.x % 3 (see row_carry_body).
-template <typename Tout, bool SEG>
-__global__ void __launch_bounds__(R_THREADS, 1)
-row_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                 const __grid_constant__ CUtensorMap tm_w,
-                 const unsigned char* __restrict__ ws, const float* __restrict__ s0,
-                 Tout* __restrict__ o, float* __restrict__ s_final, const ChunkMap m, int H,
-                 int dv, unsigned int* __restrict__ status, uint32_t spin_limit,
-                 float* __restrict__ seg_state) {
-  if constexpr (!SEG) {
-    row_carry_body<Tout, 0, false>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
-                                   spin_limit, seg_state, (int)blockIdx.x);
-  } else {
-    const int kind = (int)(blockIdx.x % 3), chain = (int)(blockIdx.x / 3);
-    if (kind == 0)
-      row_carry_body<Tout, 0, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
-                                    spin_limit, seg_state, chain);
-    else if (kind == 1)
-      row_carry_body<Tout, 1, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
-                                    spin_limit, seg_state, chain);
-    else
-      row_carry_body<Tout, 2, true>(tm_v, tm_o, tm_w, ws, s0, o, s_final, m, H, dv, status,
-                                    spin_limit, seg_state, chain);
-  }
-}
-
 }  // namespace
 
 template <typename Tout>
 cudaError_t launch_rows_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim,
-                          cudaStream_t stream, const SegmentBuffers* seg) {
+                          cudaStream_t stream) {
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
-  CUtensorMap mv, mo, mw;
+  CUtensorMap mv, mo;
   if (!encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, 32, kC, false)) return cudaErrorInvalidValue;
   const bool out_ok =
       sizeof(Tout) == 2 ? encode_bthd_bf16(&mo, a.o, TB, a.T, a.H, a.dv, a.dv, kC, false)
                         : encode_bthd_f32(&mo, (const float*)a.o, TB, a.T, a.H, a.dv, a.dv, kC);
   if (!out_ok) return cudaErrorInvalidValue;
-  const int BH = m.nseq * a.H;
-  if (seg) {
-    // two fp32 slabs of BH x [T1p tokens][128] (second-segment outputs of kinds 1 and 2)
-    if (!encode_bthd_f32(&mw, seg->outputs, 2 * BH, seg->t1p, 1, kDK, kDK, kC))
-      return cudaErrorInvalidValue;
-  } else {
-    mw = mo;   // not read
-  }
-  auto carry = seg ? row_carry_kernel<Tout, true> : row_carry_kernel<Tout, false>;
+  auto carry = row_carry_kernel<Tout>;
   cudaError_t e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, L_SMEM);
   if (e != cudaSuccess) return e;
-  carry<<<BH * (seg ? 3 : 1), R_THREADS, L_SMEM, stream>>>(
-      mv, mo, mw, (const unsigned char*)a.workspace, a.s0, (Tout*)a.o, a.s_final, m, a.H, a.dv,
-      (unsigned int*)a.workspace, lim, seg ? seg->states : nullptr);
+  carry<<<m.nseq * a.H, R_THREADS, L_SMEM, stream>>>(mv, mo, (const unsigned char*)a.workspace, a.s0,
+                                                     (Tout*)a.o, a.s_final, m, a.H, a.dv,
+                                                     (unsigned int*)a.workspace, lim);
   return cudaGetLastError();
 }
 
 cudaError_t launch_carry_rows(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
-                              cudaStream_t stream, const SegmentBuffers* seg) {
-  if (a.out_dtype == GDR_F32) return launch_rows_t<float>(a, m, spin_limit, stream, seg);
-  return launch_rows_t<__nv_bfloat16>(a, m, spin_limit, stream, seg);
+                              cudaStream_t stream) {
+  if (a.out_dtype == GDR_F32) return launch_rows_t<float>(a, m, spin_limit, stream);
+  return launch_rows_t<__nv_bfloat16>(a, m, spin_limit, stream);
 }
 
 }  // namespace gdr

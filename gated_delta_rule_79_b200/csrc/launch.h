@@ -70,26 +70,8 @@ cudaError_t launch_prefill_kda_split(const PrefillArgs& a, const ChunkMap& m,
 // (carry_sliced.cu).
 cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                                cudaStream_t stream);
-// Workspace areas of the two-segment carry (carry_rows.cu with nseg = 2, then
-// carry_segfix.cu): 3 x BH fp32 states of 128 x 128 (the first segment's final state, the
-// second segment's from zero, the transposed transition of the second segment), and two
-// fp32 slabs of BH x [t1p][128] (the second segment's outputs from zero and through the
-// identity rows); t1p = 64 x the second segment's chunks.
-struct SegmentBuffers {
-  float* states;
-  float* outputs;
-  int t1p;
-};
 cudaError_t launch_carry_rows(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
-                              cudaStream_t stream, const SegmentBuffers* seg = nullptr);
-// After launch_carry_rows with `seg`: the second segment's outputs and the final states.
-cudaError_t launch_segment_fixup(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
-                                 cudaStream_t stream, const SegmentBuffers& seg);
-// Bytes of the SegmentBuffers areas for a dense B x H batch of T tokens (0 if the
-// two-segment carry does not serve these sizes: more than kSegMaxChains chains, whose
-// three CTAs each would not fit one wave of a B200's 148 SMs, or a single chunk).
-constexpr int kSegMaxChains = 49;
-size_t segment_workspace_bytes(int B, int T, int H);
+                              cudaStream_t stream);
 cudaError_t launch_carry_sliced(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                                 cudaStream_t stream);
 size_t chunk_image_bytes();

@@ -633,10 +633,7 @@ size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
   a.dv = dv;
   a.kda = kda;
   if (!tc_prefill_supported(a)) return 0;
-  // the chunk images of the two-kernel path, then the two-segment carry's buffers (when
-  // it may serve these sizes; a workspace without them runs the other carries)
-  return (kda ? kda_split_workspace(B, T, H) : split_prefill_workspace(B, T, H)) +
-         segment_workspace_bytes(B, T, H);
+  return kda ? kda_split_workspace(B, T, H) : split_prefill_workspace(B, T, H);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {

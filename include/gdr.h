@@ -89,12 +89,9 @@ GDR_API const char* gdr_last_error(void);
  * invalid.  The workspace holds the device status word of the bounded waits
  * (the first 256 bytes) and, for the bf16 two-kernel prefills (d_k = 128, d_v a
  * multiple of 32), the precomputed operands of every chunk of 64 tokens per
- * (sequence, head): 128.5 KB per chunk for either mixer; for at most 49 (sequence,
- * head) chains it adds the buffers of the two-segment state carry (3 x 64 KB per chain
- * plus 1 KB per token of a chain's second half).  Any workspace of at least 256 bytes
- * is accepted: with less than the chunk operands the single-kernel tensor-core path
- * runs (slower; it needs the status word only), with the chunk operands but not the
- * two-segment buffers the two-kernel path runs with its other carries.  It must be
+ * (sequence, head): 128.5 KB per chunk for either mixer.  Any workspace of at least
+ * 256 bytes is accepted: with less than the returned size the single-kernel
+ * tensor-core path runs (slower; it needs the status word only).  It must be
  * zero-filled once when allocated; the library leaves it ready for the next call. */
 GDR_API size_t gdr_prefill_workspace_bytes(int B, int T, int H, int dk, int dv, int kda);
 

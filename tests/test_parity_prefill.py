@@ -317,41 +317,3 @@ def test_prefill_bf16_out_repeated(mixer):
         check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], f"{mixer} bf16 call {it}",
               bf16_out=o.dtype == torch.bfloat16)
         s_ref = to_np(state).astype(np.float64)
-
-
-@pytest.mark.parametrize("mixer", ["gdn", "kda"])
-@pytest.mark.parametrize("dv", [128, 64, 32])
-@pytest.mark.parametrize("gates", ["slow", "zero_some", "one"])
-@pytest.mark.parametrize("T,init", [(200, True), (1100, False), (130, True)])
-def test_two_segment_carry(mixer, dv, gates, T, init, monkeypatch):
-    """The two-segment carry, forced: each chain's chunks in two halves (the second run
-    from zero and through identity state rows), then the fix-up adds the first half's
-    state.  Odd and even chunk counts, ragged tails, with and without an entering state,
-    gates that keep the state alive across the halves (alpha = 1 included)."""
-    monkeypatch.setenv("GDR_CARRY", "seg")
-    w = Workload("seg", mixer, 2, 3, T, 128, dv, "bf16", "randn")
-    x = make_inputs(w, seed=T + dv + 7, gates=gates)
-    if not init:
-        x["s0"] = None
-    o, s = gpu_prefill(mixer, x, out_dtype=torch.float32)
-    o_ref, s_ref = ref_prefill(x)
-    check(o, s, o_ref, s_ref, TOL["bf16"], f"two-segment {mixer} dv={dv} gates={gates} T={T}")
-
-
-@pytest.mark.parametrize("mixer", ["gdn", "kda"])
-def test_two_segment_carry_bf16_out_in_place(mixer, monkeypatch):
-    """bf16 outputs (rounded once, after the fix-up) and the final state over the
-    entering one."""
-    import gated_delta_rule_79_b200 as g
-    monkeypatch.setenv("GDR_CARRY", "seg")
-    w = Workload("seg16", mixer, 1, 5, 1000, 128, 128, "bf16", "randn")
-    x = make_inputs(w, seed=23, gates="slow")
-    o_ref, s_ref = ref_prefill(x)
-    t = {k: v.cuda() for k, v in x.items()}
-    fn = g.kda_prefill if mixer == "kda" else g.gdn_prefill
-    state = t["s0"].clone()
-    o, s = fn(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, s_final=state)
-    torch.cuda.synchronize()
-    assert o.dtype == torch.bfloat16
-    check(to_np(o), to_np(state), o_ref, s_ref, TOL["bf16"], "two-segment bf16 in place",
-          bf16_out=True)
