@@ -25,26 +25,7 @@ struct ChunkMap {
   int nck;             // global chunks per head: B * nchunks, or an upper bound (packed)
   size_t img_base;     // byte offset of the first chunk image in the workspace
   unsigned int* checks;  // GDR_CHECKS build: the device word failed index checks set
-  int c_begin;         // dense: the part of every sequence a launch covers, chunks
-  int c_count;         //   [c_begin, c_begin + c_count) (c_count 0: all nchunks)
 };
-
-// Chunks of every sequence a launch over a dense map covers.
-__host__ __device__ __forceinline__ int part_chunks(const ChunkMap& m) {
-  return m.c_count > 0 ? m.c_count : m.nchunks;
-}
-
-// Chunk slots per head of a prep launch over this map (its grid is H times this).
-__host__ __device__ __forceinline__ int prep_slots(const ChunkMap& m) {
-  return m.cu ? m.nck : m.nseq * part_chunks(m);
-}
-
-// Global chunk of prep slot i.
-__device__ __forceinline__ int prep_slot_chunk(const ChunkMap& m, int i) {
-  if (m.cu) return i;
-  const int pc = part_chunks(m);
-  return (i / pc) * m.nchunks + m.c_begin + i % pc;
-}
 
 struct ChunkLoc {
   int seq;    // sequence
@@ -111,8 +92,8 @@ __device__ __forceinline__ void chunk_range(const ChunkMap& m, int seq, int& fir
   }
 #endif
   if (!m.cu) {
-    first = seq * m.nchunks + m.c_begin;
-    count = part_chunks(m);
+    first = seq * m.nchunks;
+    count = m.nchunks;
   } else {
     first = m.cstart[seq];
     count = m.cstart[seq + 1] - first;

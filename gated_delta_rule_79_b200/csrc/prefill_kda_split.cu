@@ -111,9 +111,8 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, hw = warp >> 2;
-  const int np = prep_slots(m);
-  const int gc = prep_slot_chunk(m, blockIdx.x % np);
-  const int h = blockIdx.x / np;
+  const int gc = blockIdx.x % m.nck;
+  const int h = blockIdx.x / m.nck;
   if (!dcheck(h < H, m.checks, kCheckImage)) return;
   const ChunkLoc loc = chunk_locate(m, gc);
   if (!loc.valid) return;            // past the last chunk of the packed sequences
@@ -421,7 +420,7 @@ cudaError_t launch_kda_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStre
              : a.pro == 1 ? kda_chunk_prep_kernel<1> : kda_chunk_prep_kernel<0>;
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  prep<<<a.H * prep_slots(m), P_THREADS, P_SMEM, stream>>>(
+  prep<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
       mq, mk, ma, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.beta,
       (unsigned char*)a.workspace, m, a.H, (unsigned int*)a.workspace, lim);
   e = cudaGetLastError();

@@ -23,8 +23,6 @@
 #include <math.h>
 #include <stdlib.h>
 
-#include <mutex>
-
 #include "gdn_prep.cuh"
 #include "launch.h"
 #include "tma_host.h"
@@ -47,9 +45,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
   unsigned char* sm = smem_raw + padb;
   PrepSmall& ps = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
   const int tid = threadIdx.x;
-  const int np = prep_slots(m);
-  const int gc = prep_slot_chunk(m, blockIdx.x % np);
-  const int h = blockIdx.x / np;
+  const int gc = blockIdx.x % m.nck;
+  const int h = blockIdx.x / m.nck;
   if (!dcheck(h < H, m.checks, kCheckImage)) return;
   if (!chunk_locate(m, gc).valid) return;   // past the last chunk of the packed sequences
   if (tid == 0) prep_init(ps);
@@ -71,36 +68,6 @@ uint32_t split_spin_limit() {
   return (uint32_t)strtoul(e, nullptr, 10);
 }
 
-// The side stream of the pipelined prefill on each device (lowest priority, so that the
-// carry's CTAs are scheduled first), created on first use.
-cudaStream_t side_stream() {
-  static std::mutex mu;
-  static cudaStream_t streams[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev]) {
-    int lo = 0, hi = 0;
-    cudaDeviceGetStreamPriorityRange(&lo, &hi);
-    cudaStream_t st = nullptr;
-    if (cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, lo) != cudaSuccess) return nullptr;
-    streams[dev] = st;
-  }
-  return streams[dev];
-}
-
-// The carry takes the value-sliced form for few long chains (carry_dispatch.cu); this
-// mirrors its rule so the pipelined prefill is used exactly when that carry runs.
-bool sliced_carry_expected(const PrefillArgs& a, const ChunkMap& m) {
-  const char* pick = getenv("GDR_CARRY");
-  if (pick && pick[0] == 'r') return false;
-  if (pick && pick[0] == 's') return true;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return (long)m.nseq * a.H * (a.dv / 32) <= sms;
-}
-
 cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t stream) {
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
@@ -113,62 +80,13 @@ cudaError_t launch_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStream_t
              : a.pro == 1 ? gdn_chunk_prep_kernel<1> : gdn_chunk_prep_kernel<0>;
   cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (e != cudaSuccess) return e;
-  auto launch_prep = [&](const ChunkMap& mm, cudaStream_t st) {
-    prep<<<a.H * prep_slots(mm), P_THREADS, P_SMEM, st>>>(
-        mq, mk, a.alpha, a.beta, (unsigned char*)a.workspace, mm, a.H,
-        (unsigned int*)a.workspace, lim);
-    return cudaGetLastError();
-  };
-
-  // Pipelined form (a dense batch on the value-sliced carry, whose few CTAs leave the SMs
-  // mostly idle while they wait on their chains): the chunks of every sequence in kParts
-  // consecutive parts; part k's carry runs while the prep of part k + 1, on a side stream,
-  // fills the room beside it.  The state passes from part to part through the
-  // workspace's state area, which follows the chunk images.
-  constexpr int kParts = 4;
-  const size_t state_off = m.img_base + (size_t)a.H * m.nck * img::kChunkWs;
-  const size_t state_bytes = (size_t)m.nseq * a.H * a.dv * kDK * sizeof(float);
-  const char* pe = getenv("GDR_PIPELINE");
-  const bool pipe = !m.cu && m.nchunks >= 2 * kParts && a.ws_bytes >= state_off + state_bytes &&
-                    !(pe && pe[0] == '0') && sliced_carry_expected(a, m);
-  cudaStream_t side = pipe ? side_stream() : nullptr;
-  if (!side) {
-    e = launch_prep(m, stream);
-    if (e != cudaSuccess) return e;
-    timing_mark(stream, 0);
-    return launch_chunk_carry(a, m, lim, stream);
-  }
-  float* sbuf = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) + state_off);
-  ChunkMap part[kParts];
-  for (int k = 0; k < kParts; ++k) {
-    part[k] = m;
-    part[k].c_begin = (int)((long)m.nchunks * k / kParts);
-    part[k].c_count = (int)((long)m.nchunks * (k + 1) / kParts) - part[k].c_begin;
-  }
-  cudaEvent_t ev[kParts] = {};
-  for (int k = 0; k < kParts; ++k) {
-    e = cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming);
-    if (e != cudaSuccess) break;
-  }
-  // the side stream starts behind everything the caller put on `stream` before this call
-  if (e == cudaSuccess) e = cudaEventRecord(ev[0], stream);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev[0], 0);
-  if (e == cudaSuccess) e = launch_prep(part[0], stream);
-  if (e == cudaSuccess) timing_mark(stream, 0);
-  for (int k = 0; k < kParts && e == cudaSuccess; ++k) {
-    if (k + 1 < kParts) {
-      e = launch_prep(part[k + 1], side);
-      if (e == cudaSuccess) e = cudaEventRecord(ev[k + 1], side);
-    }
-    if (e == cudaSuccess && k > 0) e = cudaStreamWaitEvent(stream, ev[k], 0);
-    if (e != cudaSuccess) break;
-    PrefillArgs pa = a;
-    pa.s0 = k == 0 ? a.s0 : sbuf;
-    pa.s_final = k + 1 == kParts ? a.s_final : sbuf;
-    e = launch_chunk_carry(pa, part[k], lim, stream);
-  }
-  for (int k = 0; k < kParts; ++k)
-    if (ev[k]) cudaEventDestroy(ev[k]);   // released once the work they mark completes
+  prep<<<a.H * m.nck, P_THREADS, P_SMEM, stream>>>(
+      mq, mk, a.alpha, a.beta, (unsigned char*)a.workspace, m, a.H,
+      (unsigned int*)a.workspace, lim);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  timing_mark(stream, 0);
+  e = launch_chunk_carry(a, m, lim, stream);
   return e;
 }
 

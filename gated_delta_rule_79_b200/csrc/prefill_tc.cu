@@ -633,10 +633,7 @@ size_t tc_prefill_workspace(int B, int T, int H, int dk, int dv, bool kda) {
   a.dv = dv;
   a.kda = kda;
   if (!tc_prefill_supported(a)) return 0;
-  // GDN: the chunk images, then a state area of 64 KB per (sequence, head) through which
-  // the pipelined form passes the state from one part of the chunks to the next
-  return kda ? kda_split_workspace(B, T, H)
-             : split_prefill_workspace(B, T, H) + (size_t)B * H * 128 * 128 * sizeof(float);
+  return kda ? kda_split_workspace(B, T, H) : split_prefill_workspace(B, T, H);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {

@@ -89,9 +89,7 @@ GDR_API const char* gdr_last_error(void);
  * invalid.  The workspace holds the device status word of the bounded waits
  * (the first 256 bytes) and, for the bf16 two-kernel prefills (d_k = 128, d_v a
  * multiple of 32), the precomputed operands of every chunk of 64 tokens per
- * (sequence, head): 128.5 KB per chunk for either mixer, and for GDN 64 KB per
- * (sequence, head) more, through which the pipelined GDN prefill passes the state
- * between parts of the chunks.  Any workspace of at least
+ * (sequence, head): 128.5 KB per chunk for either mixer.  Any workspace of at least
  * 256 bytes is accepted: with less than the returned size the single-kernel
  * tensor-core path runs (slower; it needs the status word only).  It must be
  * zero-filled once when allocated; the library leaves it ready for the next call. */
