@@ -438,22 +438,8 @@ def time_e2e(w, dev, steps, warmup, seed):
     x = device_inputs(w, dev, seed=seed + 100)
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
     if w.decode:
-        fn = g.kda_decode if w.mixer == "kda" else g.gdn_decode
-        state = x["s0"]
-        dbuf = {k: torch.empty_like(x[k][0]) for k in ("q", "k", "v", "alpha", "beta")}
-        o = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
-        o_host = torch.empty((w.T, w.B, w.H, w.dv), dtype=torch.bfloat16).pin_memory()
-        h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in dbuf) * w.T
-        d2h = o_host.numel() * 2
-
-        def step():
-            for t in range(w.T):
-                for key in dbuf:
-                    dbuf[key].copy_(host[key][t], non_blocking=True)
-                fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], state, o=o,
-                   prologue=w.prologue)
-                o_host[t].copy_(o, non_blocking=True)
-    elif w.varlen:
+        return _e2e_decode_overlapped(w, dev, steps, warmup, x, host)
+    if w.varlen:
         fn = g.kda_prefill_varlen if w.mixer == "kda" else g.gdn_prefill_varlen
         lens = varlen_lengths(w)
         total = sum(lens)
@@ -533,6 +519,72 @@ def time_e2e(w, dev, steps, warmup, seed):
     ms = a.elapsed_time(b) / steps
     return {"value": tokens(w) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
+
+
+def _e2e_decode_overlapped(w, dev, steps, warmup, x, host):
+    """Decode through the public API with pinned host buffers: every one of the w.T
+    decode calls of a step copies its token's q, k, v, gates and beta host->device and
+    its outputs device->host.  Two device buffer sets; the copies of token t+1 run on a
+    copy stream while the kernel of token t runs, and token t's outputs go back on a
+    third stream."""
+    import gated_delta_rule_79_b200 as g
+    fn = g.kda_decode if w.mixer == "kda" else g.gdn_decode
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    keys = ("q", "k", "v", "alpha", "beta")
+    state = x["s0"]
+    bufs = [{k: torch.empty_like(x[k][0]) for k in keys} for _ in range(2)]
+    outs = [torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    o_host = torch.empty((w.T, w.B, w.H, w.dv), dtype=torch.bfloat16).pin_memory()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in keys) * w.T
+    d2h = o_host.numel() * 2
+    count = [0]
+
+    def call(t):
+        i = count[0]
+        count[0] += 1
+        b = i % 2
+        if i >= 2:
+            up.wait_event(ev_done[b])          # call i-2 has read this input set
+        with torch.cuda.stream(up):
+            for k in keys:
+                bufs[b][k].copy_(host[k][t], non_blocking=True)
+            ev_in[b].record(up)
+        comp.wait_event(ev_in[b])
+        if i >= 2:
+            comp.wait_event(ev_out[b])         # call i-2's outputs have been copied out
+        d = bufs[b]
+        fn(d["q"], d["k"], d["v"], d["alpha"], d["beta"], state, o=outs[b], prologue=w.prologue)
+        ev_done[b].record(comp)
+        down.wait_event(ev_done[b])
+        with torch.cuda.stream(down):
+            o_host[t].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(down)
+
+    def run(n):
+        for _ in range(n):
+            for t in range(w.T):
+                call(t)
+        for b in range(2):
+            comp.wait_event(ev_out[b])
+
+    run(warmup)
+    torch.cuda.synchronize(dev)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    up.wait_event(a)
+    down.wait_event(a)
+    run(steps)
+    e.record(comp)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(e) / steps
+    return {"value": tokens(w) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+            "copies": "overlapped: host->device of token t+1 and device->host of token t-1 "
+                      "beside the kernel of token t, on three streams"}
 
 
 def _e2e_prefill_overlapped(w, dev, steps, warmup, x, host):
