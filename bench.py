@@ -704,6 +704,14 @@ def _oracle_slice(args):
     return time.perf_counter() - t
 
 
+_THREAD_VARS = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS",
+                "NUMEXPR_NUM_THREADS")
+
+
+def _single_thread_worker():
+    torch.set_num_threads(1)
+
+
 class OracleTimer:
     """Times the oracle on the host cores over a bounded sample of workload w: a
     spawn pool with one process per core, each running whole (batch, head) chains
@@ -730,10 +738,23 @@ class OracleTimer:
             self.tokens_per_unit = 1
             what = f"{self.t_sample} tokens"
         self.chains = [(w.name, i // w.H, i % w.H, self.t_sample) for i in range(self.cores)]
-        self.pool = mp.get_context("spawn").Pool(processes=self.cores)
+        # one thread per worker process (numpy's BLAS and torch would otherwise start a
+        # pool of their own in every worker and oversubscribe the cores)
+        saved = {k: os.environ.get(k) for k in _THREAD_VARS}
+        os.environ.update({k: "1" for k in _THREAD_VARS})
+        try:
+            self.pool = mp.get_context("spawn").Pool(processes=self.cores,
+                                                     initializer=_single_thread_worker)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
         self.pool.map(_oracle_slice, [(w.name, 0, 0, 1)] * self.cores)   # start the workers
         self.sample = (f"{self.cores} processes x {what} of {w.name} per pass, fp64 numpy "
-                       f"oracle, one spawn process per core; tokens/s = token-heads/s / H")
+                       f"oracle, one single-threaded spawn process per core; tokens/s = "
+                       f"token-heads/s / H")
 
     def tokens_per_pass(self):
         """Tokens (token-heads / H) one sampled pass processes."""
