@@ -1,6 +1,6 @@
-// Which state carry a two-kernel prefill runs (carry_sliced.cu or carry_rows.cu), and the
-// size of one chunk's operand image both read.  The timing aid's mark after the carry is
-// set here.
+// Which state carry a two-kernel prefill runs (carry_chain.cu, carry_rows.cu or
+// carry_sliced.cu), and the size of one chunk's operand image they read.  The timing
+// aid's mark after the carry is set here.
 
 #include <stdlib.h>
 
@@ -11,26 +11,25 @@
 
 namespace gdr {
 
-// The value-sliced carry while one 32-column slice per CTA still fits a single wave of
-// SMs (a few long chains: several SMs share each head), else the per-head carry (it
-// spends a quarter of the SM time per chunk).  GDR_CARRY=rows or GDR_CARRY=sliced picks
-// one regardless.
+// The chained carry (one CTA per (sequence, head), products fed from tensor memory) while
+// the chains fit one wave of SMs; with more chains than SMs every carry is bound by the
+// chunk images it reads, and the per-head carry takes them.  GDR_CARRY=chain, =rows or
+// =sliced picks one regardless (the value-sliced carry spreads each head over several SMs).
 cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                                cudaStream_t stream) {
   const char* pick = getenv("GDR_CARRY");
-  bool rows;
-  if (pick && pick[0] == 'r') {
-    rows = true;
-  } else if (pick && pick[0] == 's') {
-    rows = false;
+  char which;
+  if (pick && (pick[0] == 'c' || pick[0] == 'r' || pick[0] == 's')) {
+    which = pick[0];
   } else {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    rows = (long)m.nseq * a.H * (a.dv / 32) > sms;
+    which = (long)m.nseq * a.H > sms ? 'r' : 'c';
   }
-  const cudaError_t e = rows ? launch_carry_rows(a, m, spin_limit, stream)
-                             : launch_carry_sliced(a, m, spin_limit, stream);
+  const cudaError_t e = which == 'c'   ? launch_carry_chain(a, m, spin_limit, stream)
+                        : which == 'r' ? launch_carry_rows(a, m, spin_limit, stream)
+                                       : launch_carry_sliced(a, m, spin_limit, stream);
   if (e == cudaSuccess) timing_mark(stream, 1);
   return e;
 }

@@ -279,9 +279,14 @@ __device__ __forceinline__ bool prep_chunk(const CUtensorMap* tm_q, const CUtens
     const int r = tid & 63, half = tid >> 6;
     float xr[32];
 #pragma unroll
-    for (int x = 0; x < 32; ++x) {
-      const int j = half * 32 + x;
-      xr[x] = ((j >> 4) <= (r >> 4)) ? Xs[solve64::at(r, j)] * ps.beta[j] : 0.f;
+    for (int x = 0; x < 8; ++x) {
+      const int q = half * 8 + x;                    // 16-byte piece: columns 4 q .. 4 q + 3
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if ((q >> 2) <= (r >> 4)) v = *reinterpret_cast<const float4*>(Xs + solve64::at4(r, q));
+      xr[4 * x] = v.x * ps.beta[4 * q];
+      xr[4 * x + 1] = v.y * ps.beta[4 * q + 1];
+      xr[4 * x + 2] = v.z * ps.beta[4 * q + 2];
+      xr[4 * x + 3] = v.w * ps.beta[4 * q + 3];
     }
     unsigned char* it = img + img::WS_T;
 #pragma unroll

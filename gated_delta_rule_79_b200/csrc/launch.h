@@ -66,14 +66,16 @@ cudaError_t launch_prefill_kda_split(const PrefillArgs& a, const ChunkMap& m,
                                      cudaStream_t stream);
 // The state carry both two-kernel prefills share, run after the prep kernel has written
 // the chunk images; chunk_image_bytes() is the size of one image.  launch_chunk_carry
-// (carry_dispatch.cu) picks the per-head carry (carry_rows.cu) or the value-sliced one
-// (carry_sliced.cu).
+// (carry_dispatch.cu) picks the chained carry (carry_chain.cu), the per-head carry
+// (carry_rows.cu) or the value-sliced one (carry_sliced.cu).
 cudaError_t launch_chunk_carry(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                                cudaStream_t stream);
 cudaError_t launch_carry_rows(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                               cudaStream_t stream);
 cudaError_t launch_carry_sliced(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
                                 cudaStream_t stream);
+cudaError_t launch_carry_chain(const PrefillArgs& a, const ChunkMap& m, uint32_t spin_limit,
+                               cudaStream_t stream);
 size_t chunk_image_bytes();
 
 // Gradients of a dense prefill (backward.cu).

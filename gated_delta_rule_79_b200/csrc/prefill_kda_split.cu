@@ -391,11 +391,11 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       float e[4];
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (qq <= (r >> 4)) v = *reinterpret_cast<const float4*>(Xs + solve64::at4(r, 4 * qq + x));
+      const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int j = 16 * qq + 4 * x + y;
-        e[y] = (qq <= (r >> 4)) ? Xs[solve64::at(r, j)] * ps.beta[j] : 0.f;
-      }
+      for (int y = 0; y < 4; ++y) e[y] = vv[y] * ps.beta[16 * qq + 4 * x + y];
       *reinterpret_cast<float4*>(it + swz_off4(r, 4 * qq + x, 64)) = tf32x4(e[0], e[1], e[2], e[3]);
     }
   }
@@ -426,9 +426,7 @@ cudaError_t launch_kda_split_t(const PrefillArgs& a, const ChunkMap& m, cudaStre
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   timing_mark(stream, 0);
-  e = launch_chunk_carry(a, m, lim, stream);
-  e = cudaGetLastError();
-  return e;
+  return launch_chunk_carry(a, m, lim, stream);
 }
 
 }  // namespace

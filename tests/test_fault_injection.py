@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
-@pytest.mark.parametrize("path", ["single-kernel", "two-kernel rows", "two-kernel sliced"])
+@pytest.mark.parametrize("path", ["single-kernel", "two-kernel chain", "two-kernel rows",
+                                  "two-kernel sliced"])
 def test_bounded_wait_reports_timeout_and_recovers(mixer, path, monkeypatch):
     import gated_delta_rule_79_b200 as g
     if path.startswith("two-kernel"):

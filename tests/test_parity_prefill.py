@@ -231,14 +231,14 @@ def test_kda_carry_with_64_value_columns(dv, monkeypatch):
     check(o, s, o_ref, s_ref, TOL["bf16"], f"kda 64-column carry dv={dv}")
 
 
-@pytest.mark.parametrize("carry", ["rows", "sliced"])
+@pytest.mark.parametrize("carry", ["chain", "rows", "sliced"])
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
 @pytest.mark.parametrize("dv", [128, 64, 32])
 @pytest.mark.parametrize("gates", ["slow", "zero_some"])
 def test_both_carries(carry, mixer, dv, gates, monkeypatch):
-    """Either state carry, forced (the per-head one runs all value rows of a head in one
-    CTA, the value-sliced one spreads them): a ragged tail, an entering state, gates
-    that make the carry matter."""
+    """Each state carry, forced (the chained and the per-head ones run all value rows of
+    a head in one CTA, the value-sliced one spreads them): a ragged tail, an entering
+    state, gates that make the carry matter."""
     monkeypatch.setenv("GDR_CARRY", carry)
     w = Workload("carry", mixer, 2, 3, 200, 128, dv, "bf16", "randn")
     x = make_inputs(w, seed=dv + 11, gates=gates)
@@ -247,7 +247,7 @@ def test_both_carries(carry, mixer, dv, gates, monkeypatch):
     check(o, s, o_ref, s_ref, TOL["bf16"], f"{carry} carry {mixer} dv={dv} gates={gates}")
 
 
-@pytest.mark.parametrize("carry", ["rows", "sliced"])
+@pytest.mark.parametrize("carry", ["chain", "rows", "sliced"])
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
 def test_both_carries_bf16_out_in_place(carry, mixer, monkeypatch):
     """bf16 outputs and the final state written over the entering one."""

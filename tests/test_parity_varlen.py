@@ -41,7 +41,7 @@ def _run(mixer, x, cu, pool, slots, out_dtype=None):
     return o
 
 
-@pytest.mark.parametrize("carry", ["rows", "sliced"])
+@pytest.mark.parametrize("carry", ["chain", "rows", "sliced"])
 @pytest.mark.parametrize("mixer", ["gdn", "kda"])
 @pytest.mark.parametrize("dv", [128, 32])
 def test_varlen_ragged(mixer, dv, carry, monkeypatch):
