@@ -24,13 +24,16 @@
 // then accumulates onto) while the R and O products read S_c, and store the outputs.  The
 // two output products fill the tensor pipe while the issuing warp waits for R and U.
 //
-// Roles: warps 0-3 the chain's per-element passes (V^T preload, decayed state copy; value
-// row = lane of the warp's sub-partition), warps 4-7 the outputs, warp 8 the loader (bulk
-// copies of the chunk images, the V tiles by TMA, L2 prefetch two chunks ahead), warp 9
-// the issuing warp.  [Q~; K~] and e^{G_last} are double-buffered; T, V, and K^ | P have
-// one buffer each, refilled as soon as what reads them has completed.  The outputs leave
-// through shared memory, one TMA tensor store per chunk (scattered 2-byte stores from every
-// thread cost several times more).
+// Roles: warps 0-3 write the decayed state copy and the outputs (value row = lane of the
+// warp's sub-partition), warps 4-7 preload V^T (from V columns they read from global
+// memory a chunk ahead), warp 8 the loader (bulk copies of the chunk images;
+// L2 prefetch of the images and the V tiles two chunks ahead), warp 9 the issuing warp.
+// [Q~; K~] with e^{G_last}, and T are double-buffered; K^ and P have one buffer each,
+// refilled as soon as the product that reads it has completed.  The outputs leave through
+// shared memory, one TMA tensor store per chunk (scattered 2-byte stores from every
+// thread cost several times more).  The issuing warp tests every barrier a step needs at
+// once, with non-blocking tests (one blocking wait after another cost ~150-200 cycles
+// each, ten times a chunk, even when the phase had long completed).
 //
 // Precision: kind::tf32 products.  The B operands were rounded to tf32 by the prep; the A
 // operands are fp32 accumulators, of which the tensor cores use the tf32 part (the lower
@@ -64,19 +67,19 @@ constexpr int kPrefetch = GDR_CHAIN_PREFETCH;   // chunks the loader prefetches 
 constexpr int K_THREADS = 320;       // warps 0-7 per-element passes, 8 loader, 9 issuer
 constexpr int K_LANES = 256;
 
-// Shared memory: the [Q~; K~] tiles twice, T, K^ | P, V (bf16 [64 t][32 v] blocks: one
-// TMA box per 32 value columns, which lands sooner than a single box of 64 long rows),
-// e^{G_last} twice, the barriers, and the 16 KB output staging tile.
+// Shared memory: the [Q~; K~] tiles twice, T twice, K^, P, e^{G_last} twice, the barriers,
+// and the 16 KB output staging tile.  (V never passes through shared memory: the chain
+// warps read it from global memory a chunk ahead.)
 constexpr int K_A0 = 0;
 constexpr int K_A1 = WS_EGL;                  // 64 KB
-constexpr int K_T = 2 * WS_EGL;
-constexpr int K_D = K_T + 16384;
-constexpr int K_V = K_D + WS_D_BYTES;
-constexpr int K_EGL = K_V + 16384;
+constexpr int K_T = 2 * WS_EGL;               // 16 KB each
+constexpr int K_KH = K_T + 2 * 16384;         // 32 KB
+constexpr int K_P = K_KH + 32768;             // 16 KB
+constexpr int K_EGL = K_P + 16384;
 constexpr int K_SMALL = K_EGL + 1024;
 constexpr int K_STAGE = K_SMALL + 256;
 constexpr int K_SMEM = K_STAGE + 16384 + 1024;
-static_assert(K_A1 % 1024 == 0 && K_T % 1024 == 0 && K_D % 1024 == 0 && K_V % 128 == 0,
+static_assert(K_A1 % 1024 == 0 && K_T % 1024 == 0 && K_KH % 1024 == 0 && K_P % 1024 == 0,
               "tile alignment");
 static_assert(K_STAGE % 128 == 0, "TMA store source");
 static_assert(K_SMEM <= 232448, "shared memory");
@@ -88,9 +91,9 @@ constexpr uint32_t T_S = 0, T_O = 256, T_R = 384, T_U = 448, T_COLS = 512;
 struct ChainSmall {
   unsigned long long full_a[2];   // [Q~; K~] and e^{G_last} buffer has landed
   unsigned long long empty_a[2];  // ... and its readers are done (products + decay pass)
-  unsigned long long full_t, empty_t;
-  unsigned long long full_v, empty_v;
-  unsigned long long full_d, empty_d;
+  unsigned long long full_t[2], empty_t[2];
+  unsigned long long full_k, empty_k;   // K^
+  unsigned long long full_p, empty_p;   // P
   unsigned long long r_done;      // the R^T product has completed
   unsigned long long u_done;      // the U^T product has completed (R^T is free)
   unsigned long long s_done;      // the state product has completed
@@ -105,6 +108,45 @@ struct ChainSmall {
 };
 static_assert(sizeof(ChainSmall) <= 256, "small area");
 
+// V of chunk gc for the lane pair of value column v: the even lane reads columns
+// (v & ~1, v | 1) of tokens 2i, the odd lane of tokens 2i + 1, 4 bytes a load, zero past
+// the chunk's length or past d_v.  Only the loads are issued here; vcol_pairs() swaps the
+// halves between the pair once the data is needed, so the loads stay in flight meanwhile.
+__device__ __forceinline__ void fetch_v(uint32_t (&raw)[GDR_CHUNK / 2],
+                                        const __nv_bfloat16* __restrict__ vin,
+                                        const ChunkMap& m, int gc, int H, int h, int dv, int v) {
+  const ChunkLoc l = chunk_locate(m, gc);
+  const int odd = v & 1, vb = v & ~1;
+  const int n = vb < dv ? l.L : 0;      // tokens of the chunk to read
+  const __nv_bfloat16* p = vin + (((long)l.b * m.T + l.t0 + odd) * H + h) * (long)dv + vb;
+  const long ts2 = 2L * H * dv;
+#pragma unroll
+  for (int i = 0; i < GDR_CHUNK / 2; ++i) {
+    raw[i] = 2 * i + odd < n ? __ldg(reinterpret_cast<const unsigned int*>(p)) : 0u;
+    p += ts2;
+  }
+}
+// Word i of column v: bf16 of tokens 2i (low half) and 2i + 1 (high half).  All 32 lanes
+// of the warp take part.
+__device__ __forceinline__ uint32_t vcol_pair(uint32_t raw, int v) {
+  const uint32_t o = __shfl_xor_sync(0xffffffffu, raw, 1);
+  return (v & 1) ? __byte_perm(o, raw, 0x7632) : __byte_perm(raw, o, 0x5410);
+}
+
+// Non-blocking test of an mbarrier phase (no suspension, so tests of several barriers
+// issued back to back overlap their latency).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 template <typename Tout>
 __device__ __forceinline__ Tout out_cast(float x);
 template <>
@@ -116,7 +158,8 @@ __device__ __forceinline__ __nv_bfloat16 out_cast<__nv_bfloat16>(float x) {
 
 template <typename Tout>
 __global__ void __launch_bounds__(K_THREADS, 1)
-chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+chain_carry_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_v,
+                   const __nv_bfloat16* __restrict__ vin,
                    const unsigned char* __restrict__ ws,
                    const float* __restrict__ s0, Tout* __restrict__ o,
                    float* __restrict__ s_final, const ChunkMap m, int H, int dv,
@@ -127,12 +170,12 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
   ChainSmall& cs = *reinterpret_cast<ChainSmall*>(sm + K_SMALL);
   uint64_t* full_a = reinterpret_cast<uint64_t*>(&cs.full_a[0]);
   uint64_t* empty_a = reinterpret_cast<uint64_t*>(&cs.empty_a[0]);
-  uint64_t* full_t = reinterpret_cast<uint64_t*>(&cs.full_t);
-  uint64_t* empty_t = reinterpret_cast<uint64_t*>(&cs.empty_t);
-  uint64_t* full_v = reinterpret_cast<uint64_t*>(&cs.full_v);
-  uint64_t* empty_v = reinterpret_cast<uint64_t*>(&cs.empty_v);
-  uint64_t* full_d = reinterpret_cast<uint64_t*>(&cs.full_d);
-  uint64_t* empty_d = reinterpret_cast<uint64_t*>(&cs.empty_d);
+  uint64_t* full_t = reinterpret_cast<uint64_t*>(&cs.full_t[0]);
+  uint64_t* empty_t = reinterpret_cast<uint64_t*>(&cs.empty_t[0]);
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(&cs.full_k);
+  uint64_t* empty_k = reinterpret_cast<uint64_t*>(&cs.empty_k);
+  uint64_t* full_p = reinterpret_cast<uint64_t*>(&cs.full_p);
+  uint64_t* empty_p = reinterpret_cast<uint64_t*>(&cs.empty_p);
   uint64_t* r_done = reinterpret_cast<uint64_t*>(&cs.r_done);
   uint64_t* u_done = reinterpret_cast<uint64_t*>(&cs.u_done);
   uint64_t* s_done = reinterpret_cast<uint64_t*>(&cs.s_done);
@@ -148,7 +191,6 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
   int first = 0, nchunks = 0;
   chunk_range(m, seq, first, nchunks);
   if (!dcheck(dv <= 128 && dv % 32 == 0, m.checks, kCheckImage)) nchunks = 0;
-  const int nvb = dv / 32;           // TMA boxes of 32 value columns
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -156,13 +198,13 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
       mbar_init(empty_a + b, 2);     // the products' commit and the decay pass
       mbar_init(out_full + b, 1);
       mbar_init(out_free + b, 1);
+      mbar_init(full_t + b, 1);
+      mbar_init(empty_t + b, 1);
     }
-    mbar_init(full_t, 1);
-    mbar_init(empty_t, 1);
-    mbar_init(full_v, 1);
-    mbar_init(empty_v, 1);
-    mbar_init(full_d, 1);
-    mbar_init(empty_d, 1);
+    mbar_init(full_k, 1);
+    mbar_init(empty_k, 1);
+    mbar_init(full_p, 1);
+    mbar_init(empty_p, 1);
     mbar_init(r_done, 1);
     mbar_init(u_done, 1);
     mbar_init(s_done, 1);
@@ -188,32 +230,40 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
     // each product (the warp-collective form keeps the operands in uniform registers: a
     // product issues in about half the time a lone thread takes).
     {
-      const uint64_t dT = sdesc(sbase_u + K_T, 16, 1024);
-      const uint64_t dKH = sdesc(sbase_u + K_D, 16, 1024);
-      const uint64_t dP = sdesc(sbase_u + K_D + 32768, 16, 1024);
+      const uint64_t dKH = sdesc(sbase_u + K_KH, 16, 1024);
+      const uint64_t dP = sdesc(sbase_u + K_P, 16, 1024);
       const uint32_t i64 = idesc_tf32(128, 64, false, false);
       const uint32_t i64n = idesc_tf32(128, 64, false, false, true);   // -A
       const uint32_t i128 = idesc_tf32(128, 128, false, false);
       bool any = false;
-      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-        if (__all_sync(0xffffffffu, mbar_wait(bar, parity, spin_limit))) return true;
+      // Each wait point tests all the barriers it needs together, warp-uniformly, until
+      // all have completed or the limit is reached (then the give-up is recorded).
+      auto spin = [&](auto&& ready) -> bool {
+        for (uint32_t i = 0; i < spin_limit; ++i)
+          if (__all_sync(0xffffffffu, ready())) return true;
         if (lane == 0) {
           atomicOr(status, 1u);
           cs.abort = 1;
         }
         return false;
       };
-      bool ok = nchunks == 0 || wait(s0_ready, 0);
+      auto done = [&](uint64_t* bar, uint32_t parity, bool need) -> bool {
+        return !need || mbar_test(bar, parity);
+      };
+      bool ok = nchunks == 0 || spin([&] { return done(s0_ready, 0, true); });
       for (int c = 0; c < nchunks && ok && !__any_sync(0xffffffffu, *abort_flag != 0); ++c) {
         const int b = c & 1;
         const uint32_t pc = (uint32_t)c & 1u, pb = (uint32_t)(c >> 1) & 1u;
         const uint32_t tS = T_S + 128u * b, tSn = T_S + 128u * (b ^ 1), tO = T_O + 64u * b;
         const uint32_t sa = sbase_u + (b ? K_A1 : K_A0);
         const uint64_t dQ = sdesc(sa, 16, 1024), dK = sdesc(sa + 64 * 128, 16, 1024);
+        const uint64_t dT = sdesc(sbase_u + K_T + 16384 * b, 16, 1024);
         // S_c complete (the previous state product), V^T preloaded, the chunk's [Q~; K~]
         // landed, and this O^T buffer read out (chunk c - 2)
-        ok = (c == 0 || wait(s_done, pc ^ 1u)) && wait(v_ready, pc) && wait(full_a + b, pb) &&
-             (c < 2 || wait(out_free + b, pb ^ 1u));
+        ok = spin([&] {
+          return done(s_done, pc ^ 1u, c > 0) & done(v_ready, pc, true) &
+                 done(full_a + b, pb, true) & done(out_free + b, pb ^ 1u, c >= 2);
+        });
         if (!ok) break;
         fence_after_sync();
         // ---- R^T = V^T - S_c K~^T, then the first half of O^T = S_c Q~^T ----------------------
@@ -225,7 +275,7 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         for (int ks = 0; ks < kDK / 16; ++ks)
           mma_tf32_ta_w(tb + tO, tb + tS + 8 * ks, kstep(dQ, 128, ks), i64, ks > 0);
         any = true;
-        ok = wait(r_done, pc) && wait(full_t, pc);
+        ok = spin([&] { return done(r_done, pc, true) & done(full_t + b, pb, true); });
         if (!ok) break;
         fence_after_sync();
         // ---- U^T = R^T T^T, then the second half of O^T = S_c Q~^T ------------------------
@@ -233,12 +283,14 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         for (int ks = 0; ks < kC / 8; ++ks)
           mma_tf32_ta_w(tb + T_U, tb + T_R + 8 * ks, kstep(dT, 64, ks), i64, ks > 0);
         mma_commit_w(u_done);
-        mma_commit_w(empty_t);
+        mma_commit_w(empty_t + b);
 #pragma unroll
         for (int ks = kDK / 16; ks < kDK / 8; ++ks)
           mma_tf32_ta_w(tb + tO, tb + tS + 8 * ks, kstep(dQ, 128, ks), i64, true);
         mma_commit_w(empty_a + b);
-        ok = wait(u_done, pc) && wait(full_d, pc) && wait(d_ready, pc);
+        ok = spin([&] {
+          return done(u_done, pc, true) & done(full_k, pc, true) & done(d_ready, pc, true);
+        });
         if (!ok) break;
         fence_after_sync();
         // ---- S_{c+1} = S_c Diag(e^{G_last}) + U^T K^^T, then O^T += U^T P^T ---------------
@@ -246,10 +298,13 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         for (int ks = 0; ks < kC / 8; ++ks)
           mma_tf32_ta_w(tb + tSn, tb + T_U + 8 * ks, kstep(dKH, 128, ks), i128, true);
         mma_commit_w(s_done);
+        mma_commit_w(empty_k);
+        if (!(ok = spin([&] { return done(full_p, pc, true); }))) break;
+        fence_after_sync();
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
           mma_tf32_ta_w(tb + tO, tb + T_U + 8 * ks, kstep(dP, 64, ks), i64, true);
-        mma_commit_w(empty_d);
+        mma_commit_w(empty_p);
         mma_commit_w(out_full + b);
       }
       // the products issued here complete before tensor memory is freed
@@ -261,8 +316,9 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
   } else if (warp == 8) {
     // ================================ loader ===========================================
     if (lane == 0) {
-      bool issued_a[2] = {false, false}, issued_t = false, issued_v = false, issued_d = false;
-      uint32_t last_a[2] = {0, 0}, last_t = 0, last_v = 0, last_d = 0;
+      bool issued_a[2] = {false, false}, issued_t[2] = {false, false}, issued_k = false,
+           issued_p = false;
+      uint32_t last_a[2] = {0, 0}, last_t[2] = {0, 0}, last_k = 0, last_p = 0;
       auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
         if (mbar_wait(bar, parity, spin_limit)) return true;
         atomicOr(status, 1u);
@@ -273,59 +329,59 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         const unsigned char* src = wsb + (size_t)c * kChunkWs;
         const int b = c & 1;
         const uint32_t pc = (uint32_t)c & 1u, pb = (uint32_t)(c >> 1) & 1u;
-        const ChunkLoc loc = chunk_locate(m, first + c);
-        // in the order their buffers free up: [Q~; K~] (chunk c - 2's), V, T, K^ | P
+        // in the order their buffers free up: [Q~; K~] and T (chunk c - 2's), K^, P
         if (!wait(empty_a + b, pb ^ 1u)) break;
         mbar_expect_tx(full_a + b, WS_A_BYTES);
         bulk_load(sbase_u + (b ? K_A1 : K_A0), src + WS_QK, WS_EGL, full_a + b);
         bulk_load(sbase_u + K_EGL + 512 * b, src + WS_EGL, WS_A_BYTES - WS_EGL, full_a + b);
         issued_a[b] = true;
         last_a[b] = pb;
-        if (!wait(empty_v, pc ^ 1u)) break;
-        mbar_expect_tx(full_v, (uint32_t)(nvb * 4096));
-        for (int nb = 0; nb < nvb; ++nb)
-          tma_load_4d(sbase_u + K_V + nb * 4096, &tm_v, 32 * nb, h, loc.t0, loc.b, full_v);
-        issued_v = true;
-        last_v = pc;
-        if (!wait(empty_t, pc ^ 1u)) break;
-        mbar_expect_tx(full_t, 16384);
-        bulk_load(sbase_u + K_T, src + WS_T, 16384, full_t);
-        issued_t = true;
-        last_t = pc;
-        if (!wait(empty_d, pc ^ 1u)) break;
-        mbar_expect_tx(full_d, WS_D_BYTES);
-        bulk_load(sbase_u + K_D, src + WS_KH, WS_D_BYTES, full_d);
-        issued_d = true;
-        last_d = pc;
-        // L2 prefetch kPrefetch chunks ahead (the first ones at the start)
+        if (!wait(empty_t + b, pb ^ 1u)) break;
+        mbar_expect_tx(full_t + b, 16384);
+        bulk_load(sbase_u + K_T + 16384 * b, src + WS_T, 16384, full_t + b);
+        issued_t[b] = true;
+        last_t[b] = pb;
+        if (!wait(empty_k, pc ^ 1u)) break;
+        mbar_expect_tx(full_k, 32768);
+        bulk_load(sbase_u + K_KH, src + WS_KH, 32768, full_k);
+        issued_k = true;
+        last_k = pc;
+        if (!wait(empty_p, pc ^ 1u)) break;
+        mbar_expect_tx(full_p, 16384);
+        bulk_load(sbase_u + K_P, src + WS_P, 16384, full_p);
+        issued_p = true;
+        last_p = pc;
+        // L2 prefetch kPrefetch chunks ahead (the first ones at the start): the chunk image,
+        // and the V tile that the V warps read with plain loads a chunk ahead
         for (int p = c == 0 ? 1 : kPrefetch; p <= kPrefetch && c + p < nchunks; ++p) {
           bulk_prefetch_l2(src + (size_t)p * kChunkWs, kChunkWs);
-          const ChunkLoc l2 = chunk_locate(m, first + c + p);
-          for (int nb = 0; nb < nvb; ++nb) tma_prefetch_4d(&tm_v, 32 * nb, h, l2.t0, l2.b);
+          const ChunkLoc lp = chunk_locate(m, first + c + p);
+          tma_prefetch_4d(&tm_v, 0, h, lp.t0, lp.b);
         }
       }
       {
         // copies issued here may still be landing in shared memory (after a give-up
         // anywhere): let them finish (a barrier's phases complete in order, so its last
         // copy is the one to wait for; after a normal run they all have)
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < 2; ++b) {
           if (issued_a[b]) mbar_wait(full_a + b, last_a[b], kDrainLimit);
-        if (issued_v) mbar_wait(full_v, last_v, kDrainLimit);
-        if (issued_t) mbar_wait(full_t, last_t, kDrainLimit);
-        if (issued_d) mbar_wait(full_d, last_d, kDrainLimit);
+          if (issued_t[b]) mbar_wait(full_t + b, last_t[b], kDrainLimit);
+        }
+        if (issued_k) mbar_wait(full_k, last_k, kDrainLimit);
+        if (issued_p) mbar_wait(full_p, last_p, kDrainLimit);
       }
     }
   } else {
     // ========================== per-element passes =====================================
     // Two groups of four warps, each covering all 128 value rows (warp w % 4 reaches TMEM
-    // lanes 32 (w % 4) ..): warps 0-3 keep the chain fed (V^T preload, decayed state copy,
-    // entering and final state), warps 4-7 write the outputs, so neither waits for the other.
-    const bool outg = warp >= 4;
+    // lanes 32 (w % 4) ..).  Warps 0-3 write the entering state, each chunk's decayed state
+    // copy, the outputs and the final state; warps 4-7 preload V^T and read the next
+    // chunk's V from global memory (issuing those loads stalls for a while when many are
+    // in flight, so it comes after the preload has been signalled).
+    const bool vg = warp >= 4;
     const int gid = tid & 127;
     const int v = gid;                      // value row = TMEM lane
     const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
-    const int sidx = chunk_state_index(m, seq);
-    const long srow = (((long)max(sidx, 0) * H + h) * dv + v) * kDK;
     bool fail = false;
     // a wait every thread makes; the group barrier after the pass tells all of its threads
     // whether anyone gave up (the passes only touch this CTA's shared and tensor memory, so
@@ -334,12 +390,103 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
       if (!fail && !mbar_wait(bar, parity, spin_limit)) fail = true;
     };
     auto agree = [&]() -> bool {
-      return named_bar_or(outg ? 2 : 1, K_LANES / 2, fail || *abort_flag != 0);
+      return named_bar_or(vg ? 2 : 1, K_LANES / 2, fail || *abort_flag != 0);
     };
     bool stop = false;
-    if (!outg) {
-      // ---------------------------- chain warps ----------------------------------------
-      const unsigned char* vcol = sm + K_V + (v >> 5) * 4096 + (v & 31) * 2;
+    if (vg) {
+      // ------------------------------- V warps -----------------------------------------
+      uint32_t vraw[kC / 2];
+      if (nchunks > 0) fetch_v(vraw, vin, m, first, H, h, dv, v);
+      for (int c = 0; c < nchunks && !stop; ++c) {
+        // V^T of chunk c into R^T's columns, once chunk c - 1's U^T product has read R^T
+        if (c > 0) pass_wait(u_done, (uint32_t)(c - 1) & 1u);
+        fence_after_sync();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t w = vcol_pair(vraw[16 * hh + i], v);
+            x[2 * i] = __uint_as_float(w << 16);
+            x[2 * i + 1] = __uint_as_float(w & 0xffff0000u);
+          }
+          tmem_st32(tb + tlane + T_R + 32 * hh, x);
+        }
+        tmem_wait_st();
+        fence_before_sync();
+        if ((stop = agree())) break;
+        if (gid == 0) mbar_arrive(v_ready);
+        if (c + 1 < nchunks) fetch_v(vraw, vin, m, first + c + 1, H, h, dv, v);
+      }
+    } else {
+      // --------------------------- state and output warps ------------------------------
+      const int sidx = chunk_state_index(m, seq);
+      const long srow = (((long)max(sidx, 0) * H + h) * dv + v) * kDK;
+      // O^T of chunk c: one value column of 64 tokens per thread, staged as [t][d_v] and
+      // written by one TMA tensor store per 16 KB tile (rows past the tensor's end are not
+      // written).  A packed sequence's partial last chunk, whose rows past its end belong
+      // to the next sequence, is stored element by element instead.
+      constexpr int kRounds = (int)sizeof(Tout) / 2;     // 16 KB tiles per chunk
+      unsigned char* stage = sm + K_STAGE;
+      const bool storer = gid == 0;
+      auto write_outputs = [&](int c) -> bool {
+        const int b = c & 1;
+        pass_wait(out_full + b, (uint32_t)(c >> 1) & 1u);
+        fence_after_sync();
+        const ChunkLoc loc = chunk_locate(m, first + c);
+        const bool tma = loc.valid && !(m.cu && loc.L < kC);
+        Tout* col = o + (((long)loc.b * m.T + loc.t0) * H + h) * (long)dv + v;
+        const long tstride = (long)H * dv;
+        if (tma) {
+          if (storer) bulk_wait_read_all();      // the tile's previous store has read it
+          named_bar(3, K_LANES / 2);
+        }
+        // 32 tokens at a time: bf16 outputs fill one 64-token tile, fp32 ones two tiles of
+        // 32 tokens in turn (the first stored before the second is staged)
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[32];
+          tmem_ld32(tb + tlane + T_O + 64 * b + 32 * hh, x);
+          tmem_wait_ld();
+          if (kRounds == 2 && hh == 1 && tma) {
+            if (storer) bulk_wait_read_all();
+            named_bar(3, K_LANES / 2);
+          }
+          if (loc.valid && v < dv) {
+            if (tma) {
+              const int row0 = kRounds == 2 ? 0 : 32 * hh;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                *reinterpret_cast<Tout*>(stage + ((row0 + i) * dv + v) * (int)sizeof(Tout)) =
+                    out_cast<Tout>(x[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (32 * hh + i < loc.L) col[(32 * hh + i) * tstride] = out_cast<Tout>(x[i]);
+            }
+          }
+          if (kRounds == 2 && hh == 0 && tma) {
+            fence_smem_to_async();
+            named_bar(3, K_LANES / 2);
+            if (storer) {
+              tma_store_4d(&tm_o, smem_u32(stage), 0, h, loc.t0, loc.b);
+              bulk_commit();
+            }
+          }
+        }
+        fence_smem_to_async();
+        fence_before_sync();
+        if (agree()) return false;
+        if (storer) {
+          mbar_arrive(out_free + b);
+          const int r0 = kRounds == 2 ? 32 : 0;       // the tile staged last
+          if (tma && r0 < loc.L) {
+            tma_store_4d(&tm_o, smem_u32(stage), 0, h, loc.t0 + r0, loc.b);
+            bulk_commit();
+          }
+        }
+        return true;
+      };
       // the entering state (rows past d_v zero) into state buffer 0
 #pragma unroll
       for (int nb = 0; nb < 4; ++nb) {
@@ -360,30 +507,13 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
       fence_before_sync();
       stop = agree();
       if (!stop && gid == 0) mbar_arrive(s0_ready);
-      for (int c = 0; c < nchunks && !stop; ++c) {
+      for (int c = 0; c <= nchunks && !stop; ++c) {
+        if (c == nchunks) {
+          stop = nchunks > 0 && !write_outputs(c - 1);
+          break;
+        }
         const int b = c & 1;
         const uint32_t pc = (uint32_t)c & 1u, pb = (uint32_t)(c >> 1) & 1u;
-        // ---- V^T into R^T's columns, once the previous chunk's U^T product has read R^T --
-        pass_wait(full_v, pc);
-        if (c > 0) pass_wait(u_done, pc ^ 1u);
-        fence_after_sync();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float x[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            x[i] = v < dv ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                vcol + (32 * hh + i) * 64))
-                          : 0.f;
-          tmem_st32(tb + tlane + T_R + 32 * hh, x);
-        }
-        tmem_wait_st();
-        fence_before_sync();
-        if ((stop = agree())) break;
-        if (gid == 0) {
-          mbar_arrive(v_ready);
-          mbar_arrive(empty_v);
-        }
         // ---- S_c Diag(e^{G_last}) into the other state buffer, once S_c is complete ------
         pass_wait(full_a + b, pb);
         if (c > 0) pass_wait(s_done, pc ^ 1u);
@@ -392,23 +522,19 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
           const float4* egl = reinterpret_cast<const float4*>(sm + K_EGL + 512 * b);
           const uint32_t tS = T_S + 128u * b, tSn = T_S + 128u * (b ^ 1);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float x[2][32];
-            tmem_ld32(tb + tlane + tS + 64 * hh, x[0]);
-            tmem_ld32(tb + tlane + tS + 64 * hh + 32, x[1]);
+          for (int nb = 0; nb < 4; ++nb) {
+            float x[32];
+            tmem_ld32(tb + tlane + tS + 32 * nb, x);
             tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 e = egl[16 * hh + 8 * u + q];
-                x[u][4 * q] *= e.x;
-                x[u][4 * q + 1] *= e.y;
-                x[u][4 * q + 2] *= e.z;
-                x[u][4 * q + 3] *= e.w;
-              }
-              tmem_st32(tb + tlane + tSn + 64 * hh + 32 * u, x[u]);
+            for (int q = 0; q < 8; ++q) {
+              const float4 e = egl[8 * nb + q];
+              x[4 * q] *= e.x;
+              x[4 * q + 1] *= e.y;
+              x[4 * q + 2] *= e.z;
+              x[4 * q + 3] *= e.w;
             }
+            tmem_st32(tb + tlane + tSn + 32 * nb, x);
           }
         }
         tmem_wait_st();
@@ -418,6 +544,8 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
           mbar_arrive(d_ready);
           mbar_arrive(empty_a + b);
         }
+        // ---- the previous chunk's outputs -----------------------------------------------
+        if (c > 0 && (stop = !write_outputs(c - 1))) break;
       }
       // the final state (the last state product's result, undecayed)
       if (!stop && s_final) {
@@ -438,58 +566,6 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_consta
         }
         if (fail) stop = true;
       }
-    } else {
-      // ---------------------------- output warps ---------------------------------------
-      // O^T of each chunk: one value column of 64 tokens per thread, staged as [t][d_v] and
-      // written by one TMA tensor store per 16 KB tile (rows past the tensor's end are not
-      // written).  A packed sequence's partial last chunk, whose rows past its end belong
-      // to the next sequence, is stored element by element instead.
-      constexpr int kRounds = (int)sizeof(Tout) / 2;     // 16 KB tiles per chunk
-      constexpr int kTok = 64 / kRounds;
-      unsigned char* stage = sm + K_STAGE;
-      const bool storer = gid == 0;
-      for (int c = 0; c < nchunks && !stop; ++c) {
-        const int b = c & 1;
-        pass_wait(out_full + b, (uint32_t)(c >> 1) & 1u);
-        fence_after_sync();
-        float x[64];
-        tmem_ld32(tb + tlane + T_O + 64 * b, *reinterpret_cast<float(*)[32]>(&x[0]));
-        tmem_ld32(tb + tlane + T_O + 64 * b + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-        tmem_wait_ld();
-        fence_before_sync();
-        if ((stop = agree())) break;
-        if (storer) mbar_arrive(out_free + b);
-        const ChunkLoc loc = chunk_locate(m, first + c);
-        if (!loc.valid) continue;
-        if (m.cu && loc.L < kC) {
-          if (v < dv) {
-            const long tstride = (long)H * dv;
-            Tout* col = o + (((long)loc.b * m.T + loc.t0) * H + h) * (long)dv + v;
-#pragma unroll
-            for (int t = 0; t < kC; ++t)
-              if (t < loc.L) col[t * tstride] = out_cast<Tout>(x[t]);
-          }
-          continue;
-        }
-#pragma unroll
-        for (int r = 0; r < kRounds; ++r) {
-          if (kTok * r >= loc.L) break;          // the tile starts past the tensor's end
-          if (storer) bulk_wait_read_all();      // the tile's previous store has read it
-          named_bar(3, K_LANES / 2);
-          if (v < dv) {
-#pragma unroll
-            for (int i = 0; i < kTok; ++i)
-              *reinterpret_cast<Tout*>(stage + (i * dv + v) * (int)sizeof(Tout)) =
-                  out_cast<Tout>(x[kTok * r + i]);
-          }
-          fence_smem_to_async();
-          named_bar(3, K_LANES / 2);
-          if (storer) {
-            tma_store_4d(&tm_o, smem_u32(stage), 0, h, loc.t0 + kTok * r, loc.b);
-            bulk_commit();
-          }
-        }
-      }
       if (storer) bulk_wait_all();    // the output stores read shared memory until done
     }
     if (stop && gid == 0) {
@@ -509,8 +585,9 @@ cudaError_t launch_chain_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim
                            cudaStream_t stream) {
   // packed sequences: the tensors are [1, total, H, *]
   const int TB = m.cu ? 1 : a.B;
-  CUtensorMap mv, mo;
-  if (!encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, 32, kC, false)) return cudaErrorInvalidValue;
+  CUtensorMap mo, mv;
+  // V: one box of d_v x 64 tokens, used for L2 prefetch only
+  if (!encode_bthd_bf16(&mv, a.v, TB, a.T, a.H, a.dv, a.dv, kC, false)) return cudaErrorInvalidValue;
   // output boxes of 16 KB: 64 tokens of bf16 or 32 of fp32
   const bool out_ok =
       sizeof(Tout) == 2 ? encode_bthd_bf16(&mo, a.o, TB, a.T, a.H, a.dv, a.dv, 64, false)
@@ -519,7 +596,8 @@ cudaError_t launch_chain_t(const PrefillArgs& a, const ChunkMap& m, uint32_t lim
   auto carry = chain_carry_kernel<Tout>;
   cudaError_t e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
   if (e != cudaSuccess) return e;
-  carry<<<m.nseq * a.H, K_THREADS, K_SMEM, stream>>>(mv, mo, (const unsigned char*)a.workspace,
+  carry<<<m.nseq * a.H, K_THREADS, K_SMEM, stream>>>(mo, mv, (const __nv_bfloat16*)a.v,
+                                                     (const unsigned char*)a.workspace,
                                                      a.s0, (Tout*)a.o, a.s_final, m, a.H, a.dv,
                                                      (unsigned int*)a.workspace, lim);
   return cudaGetLastError();
