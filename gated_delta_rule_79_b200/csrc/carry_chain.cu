@@ -325,17 +325,27 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_consta
         cs.abort = 1;
         return false;
       };
-      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
-        const unsigned char* src = wsb + (size_t)c * kChunkWs;
-        const int b = c & 1;
-        const uint32_t pc = (uint32_t)c & 1u, pb = (uint32_t)(c >> 1) & 1u;
-        // in the order their buffers free up: [Q~; K~] and T (chunk c - 2's), K^, P
-        if (!wait(empty_a + b, pb ^ 1u)) break;
+      // [Q~; K~] and e^{G_last} of chunk cc into buffer cc & 1 once chunk cc - 2 is done with it
+      auto load_a = [&](int cc) -> bool {
+        const unsigned char* src = wsb + (size_t)cc * kChunkWs;
+        const int b = cc & 1;
+        const uint32_t pb = (uint32_t)(cc >> 1) & 1u;
+        if (!wait(empty_a + b, pb ^ 1u)) return false;
         mbar_expect_tx(full_a + b, WS_A_BYTES);
         bulk_load(sbase_u + (b ? K_A1 : K_A0), src + WS_QK, WS_EGL, full_a + b);
         bulk_load(sbase_u + K_EGL + 512 * b, src + WS_EGL, WS_A_BYTES - WS_EGL, full_a + b);
         issued_a[b] = true;
         last_a[b] = pb;
+        return true;
+      };
+      if (nchunks > 0) load_a(0);
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const unsigned char* src = wsb + (size_t)c * kChunkWs;
+        const int b = c & 1;
+        const uint32_t pc = (uint32_t)c & 1u, pb = (uint32_t)(c >> 1) & 1u;
+        // in the order their buffers free up: [Q~; K~] one chunk further ahead (its buffer
+        // frees in the middle of chunk c - 1), T (chunk c - 2's), K^, P
+        if (c + 1 < nchunks && !load_a(c + 1)) break;
         if (!wait(empty_t + b, pb ^ 1u)) break;
         mbar_expect_tx(full_t + b, 16384);
         bulk_load(sbase_u + K_T + 16384 * b, src + WS_T, 16384, full_t + b);
