@@ -110,14 +110,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def carry_kernel(nseq, H):
-    """The state carry a two-kernel prefill of nseq sequences x H heads runs: the library's
-    own rule (GDR_CARRY overrides it), restated here to name the kernel in the report."""
+def carry_kernel():
+    """The state carry a two-kernel prefill runs: the chained one unless GDR_CARRY picks
+    another (the library's rule, restated here to name the kernel in the report)."""
     pick = os.environ.get("GDR_CARRY", "")[:1]
-    if pick not in ("c", "r", "s"):
-        sms = torch.cuda.get_device_properties(0).multi_processor_count
-        pick = "c" if nseq * H <= sms else "r"
-    return {"c": "chain_carry_kernel", "r": "row_carry_kernel", "s": "sliced_carry_kernel"}[pick]
+    return {"r": "row_carry_kernel", "s": "sliced_carry_kernel"}.get(pick, "chain_carry_kernel")
 
 
 def load_traffic(kernel_key):
@@ -270,7 +267,7 @@ class PrefillRunner:
         # the tensor-core path with a full-size workspace runs a per-chunk prep kernel,
         # then the state carry; the others run one kernel per call
         if self.path == "tensor-core":
-            self.kernels = [f"{w.mixer}_chunk_prep_kernel", carry_kernel(w.B, w.H)]
+            self.kernels = [f"{w.mixer}_chunk_prep_kernel", carry_kernel()]
             self.kernel_key = f"prefill_two-kernel:{w.name}"
         else:
             self.kernels = ["prefill_simt_kernel"]
@@ -352,7 +349,7 @@ class VarlenRunner:
                                                         int(w.mixer == "kda"))
         self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
         self.kernels = ["varlen index + " + f"{w.mixer}_chunk_prep_kernel",
-                        carry_kernel(len(lens), w.H)]
+                        carry_kernel()]
         self.launches_per_step = 3
         self.kernel_key = f"prefill_two-kernel:{w.name}"
         self.path = "tensor-core"

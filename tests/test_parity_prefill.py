@@ -266,9 +266,9 @@ def test_both_carries_bf16_out_in_place(carry, mixer, monkeypatch):
           bf16_out=True)
 
 
-def test_many_chains_take_the_per_head_carry():
-    """40 sequences x 4 heads x 4 value slices exceed the SM count, so the automatic
-    choice is the per-head carry; checked against the oracle on sampled chains."""
+def test_more_chains_than_sms():
+    """40 sequences x 4 heads = 160 chains, more than the SMs: the chained carry runs
+    them in a second wave; checked against the oracle on sampled chains."""
     w = Workload("many", "gdn", 40, 4, 96, 128, 128, "bf16", "randn")
     x = make_inputs(w, seed=31, gates="slow")
     o, s = gpu_prefill("gdn", x, out_dtype=torch.float32)
