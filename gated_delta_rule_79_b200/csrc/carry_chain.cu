@@ -22,7 +22,7 @@
 // them; the CUDA cores work beside the chain: they preload V^T for the next chunk, write
 // the decayed copy S_c Diag(e^{G_last}) into the second state buffer (which the S product
 // then accumulates onto) while the R and O products read S_c, and store the outputs.  The
-// two output products fill the tensor pipe while the issuing warp waits for R and U.
+// two output products fill the tensor pipe while the issuing warp waits for R and for S.
 //
 // Roles: warps 0-3 write the decayed state copy and the outputs (value row = lane of the
 // warp's sub-partition), warps 4-7 preload V^T (from V columns they read from global
@@ -266,28 +266,26 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_consta
         });
         if (!ok) break;
         fence_after_sync();
-        // ---- R^T = V^T - S_c K~^T, then the first half of O^T = S_c Q~^T ----------------------
+        // ---- R^T = V^T - S_c K~^T, then O^T = S_c Q~^T (which the pipe runs while the issuing
+        //      warp waits for R: measured faster than splitting it around U) ------------------
 #pragma unroll
         for (int ks = 0; ks < kDK / 8; ++ks)
           mma_tf32_ta_w(tb + T_R, tb + tS + 8 * ks, kstep(dK, 128, ks), i64n, true);
         mma_commit_w(r_done);
 #pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks)
+        for (int ks = 0; ks < kDK / 8; ++ks)
           mma_tf32_ta_w(tb + tO, tb + tS + 8 * ks, kstep(dQ, 128, ks), i64, ks > 0);
+        mma_commit_w(empty_a + b);
         any = true;
         ok = spin([&] { return done(r_done, pc, true) & done(full_t + b, pb, true); });
         if (!ok) break;
         fence_after_sync();
-        // ---- U^T = R^T T^T, then the second half of O^T = S_c Q~^T ------------------------
+        // ---- U^T = R^T T^T --------------------------------------------------------------------
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
           mma_tf32_ta_w(tb + T_U, tb + T_R + 8 * ks, kstep(dT, 64, ks), i64, ks > 0);
         mma_commit_w(u_done);
         mma_commit_w(empty_t + b);
-#pragma unroll
-        for (int ks = kDK / 16; ks < kDK / 8; ++ks)
-          mma_tf32_ta_w(tb + tO, tb + tS + 8 * ks, kstep(dQ, 128, ks), i64, true);
-        mma_commit_w(empty_a + b);
         ok = spin([&] {
           return done(u_done, pc, true) & done(full_k, pc, true) & done(d_ready, pc, true);
         });
