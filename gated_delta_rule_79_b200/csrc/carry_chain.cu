@@ -110,7 +110,7 @@ static_assert(sizeof(ChainSmall) <= 256, "small area");
 
 // V of chunk gc for the lane pair of value column v: the even lane reads columns
 // (v & ~1, v | 1) of tokens 2i, the odd lane of tokens 2i + 1, 4 bytes a load, zero past
-// the chunk's length or past d_v.  Only the loads are issued here; vcol_pairs() swaps the
+// the chunk's length or past d_v.  Only the loads are issued here; vcol_pair() swaps the
 // halves between the pair once the data is needed, so the loads stay in flight meanwhile.
 __device__ __forceinline__ void fetch_v(uint32_t (&raw)[GDR_CHUNK / 2],
                                         const __nv_bfloat16* __restrict__ vin,
