@@ -27,7 +27,8 @@
 // Roles: warps 0-3 write the decayed state copy and the outputs (value row = lane of the
 // warp's sub-partition), warps 4-7 preload V^T (from V columns they read from global
 // memory a chunk ahead), warp 8 the loader (bulk copies of the chunk images;
-// L2 prefetch of the images and the V tiles two chunks ahead), warp 9 the issuing warp.
+// L2 prefetch of the images and the V tiles a chunk ahead: two or three chunks ahead
+// measured slower with many chains), warp 9 the issuing warp.
 // [Q~; K~] with e^{G_last}, and T are double-buffered; K^ and P have one buffer each,
 // refilled as soon as the product that reads it has completed.  The outputs leave through
 // shared memory, one TMA tensor store per chunk (scattered 2-byte stores from every
@@ -61,7 +62,7 @@ constexpr int kDK = 128;
 constexpr uint32_t kDrainLimit = 1u << 26;
 
 #ifndef GDR_CHAIN_PREFETCH
-#define GDR_CHAIN_PREFETCH 2
+#define GDR_CHAIN_PREFETCH 1
 #endif
 constexpr int kPrefetch = GDR_CHAIN_PREFETCH;   // chunks the loader prefetches into L2 ahead
 constexpr int K_THREADS = 320;       // warps 0-7 per-element passes, 8 loader, 9 issuer
