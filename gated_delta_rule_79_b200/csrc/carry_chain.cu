@@ -69,8 +69,8 @@ constexpr int K_THREADS = 320;       // warps 0-7 per-element passes, 8 loader, 
 constexpr int K_LANES = 256;
 
 // Shared memory: the [Q~; K~] tiles twice, T twice, K^, P, e^{G_last} twice, the barriers,
-// and the 16 KB output staging tile.  (V never passes through shared memory: the chain
-// warps read it from global memory a chunk ahead.)
+// and the 16 KB output staging tile.  (V never passes through shared memory: warps 4-7
+// read it from global memory a chunk ahead.)
 constexpr int K_A0 = 0;
 constexpr int K_A1 = WS_EGL;                  // 64 KB
 constexpr int K_T = 2 * WS_EGL;               // 16 KB each
@@ -393,8 +393,8 @@ chain_carry_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_consta
     const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
     bool fail = false;
     // a wait every thread makes; the group barrier after the pass tells all of its threads
-    // whether anyone gave up (the passes only touch this CTA's shared and tensor memory, so
-    // a pass over stale data is harmless)
+    // whether anyone gave up (a pass over stale data touches only this CTA's shared and
+    // tensor memory and its own output rows, so it is harmless: the give-up is recorded)
     auto pass_wait = [&](uint64_t* bar, uint32_t parity) {
       if (!fail && !mbar_wait(bar, parity, spin_limit)) fail = true;
     };
