@@ -26,10 +26,14 @@ chunked     an independent fp64 chunk-wise restatement, used only to pin the
             chunk algebra against the definition
 backward    the gradients of the recurrence (inputs, gates and initial state),
             token by token in reverse
+chunked_backward
+            the same gradients from the chunk algebra (the state gradient chained
+            through the chunks in reverse), pinned against backward
 prologue    L2-normalised q, k and the gate from its logit (the fused prologue)
 """
 
 from .recurrent import gated_delta_rule, decode_step, verify_steps, prefill_varlen  # noqa: F401
 from .chunked import chunked_gated_delta_rule  # noqa: F401
 from .backward import gated_delta_rule_backward  # noqa: F401
+from .chunked_backward import chunked_gated_delta_rule_backward  # noqa: F401
 from .prologue import apply_prologue, gate_from_logit, l2_normalise  # noqa: F401
