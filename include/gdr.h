@@ -34,6 +34,17 @@
  *     prefill is 64 tokens; the last chunk of a sequence may be shorter.
  *   - The library is thread-safe for calls on different streams; calls that
  *     share a workspace must not overlap on the device.
+ *
+ * Environment variables, read at every call (neither is needed in normal use)
+ *   GDR_SPIN_LIMIT  polls of every bounded device-side wait before it gives up
+ *                   and records GDR_ERR_TIMEOUT (default 2^24; 0 gives up
+ *                   without polling, which tests use to reach that path; the
+ *                   work in flight still completes and is drained).
+ *   GDR_CARRY       state carry of the two-kernel prefill: unset (or any other
+ *                   value) = the chained carry; "rows" = one CTA per (sequence,
+ *                   head) with the output products off its chain; "sliced" = the
+ *                   value rows of each head split over several CTAs.  All three
+ *                   give results within the same tolerance; they differ in speed.
  */
 #ifndef GDR_H_
 #define GDR_H_
